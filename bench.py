@@ -1,0 +1,460 @@
+#!/usr/bin/env python
+"""Benchmark of one ragged paged attention pass (rpa_forward) on B200.
+
+A step is one rpa_forward call over one synthetic batch: the fused cache
+update, the decode / prefill kernels, the split-KV combine -- every part of
+the method.  The headline line is the 128-sequence decode batch shaped like a
+Llama-3-8B attention layer (metric: decode HBM GB/s); the prefill (causal and
+not), mixed-batch and head_dim-256 long-context workloads are measured in the
+same run and reported under "also".
+
+Timing: W untimed warm-up steps, then K steps timed on the device with CUDA
+events on the launching stream, a 256 MiB write between steps to flush the
+126 MB L2, barrier + synchronize on both sides, max over ranks.  Algorithmic
+bytes and FLOPs follow the method's minimum work: K and V of every visible
+position read once, the new K/V written once, Q read and out / lse written
+once, the page-table entries read once; FLOPs count visible (q, k) pairs only.
+
+``--impl reference`` times the fp64 CPU oracle instead, on a bounded sample
+of the same workload (the only other place this script runs the oracle).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from ragged_paged_attention_03_b200 import inputs as I  # noqa: E402
+
+FLUSH_BYTES = 256 << 20
+WORKLOAD_TEXT = {
+    "decode_128": "decode: 128 seqs, q_len 1, kv_len U[1024,8192], Hq 32 / Hkv 8, D 128, page 16, "
+                  "bf16, 0.5*N(0,1), shuffled 1.25x page pool",
+    "prefill_8x2048": "prefill: 8 fresh seqs q_len = kv_len = 2048, Hq 32 / Hkv 8, D 128, page 16, "
+                      "bf16, N(0,1), shuffled 1.25x pool",
+    "mixed_96d_4c": "mixed: 96 decode seqs kv log-U[512,16384] + 4 chunked seqs q_len 512 after "
+                    "log-U[1024,8192] context, Hq 32 / Hkv 8, D 128, page 16, bf16, causal",
+    "long_d256": "long context: 32 decode seqs kv 131072 + 4 prefill seqs 4096, Hq 16 / Hkv 4, "
+                 "D 256, page 64, bf16, causal",
+}
+
+
+# ------------------------------------------------------------ work counting
+def algorithmic(prob: I.Problem) -> dict:
+    """Minimum bytes and FLOPs of one pass (see module docstring)."""
+    e = 4 if prob.dtype == I.F32 else 2
+    hq, hkv, d, p = prob.num_q_heads, prob.num_kv_heads, prob.head_dim, prob.page_size
+    q = prob.q_lens.astype(np.int64)
+    k = prob.kv_lens.astype(np.int64)
+    t = int(q.sum())
+    kv_read = int(k.sum()) * hkv * d * 2 * e
+    cache_write = t * hkv * d * 2 * e
+    q_out = 2 * t * hq * d * e
+    lse = 4 * t * hq
+    table = 4 * int(((k + p - 1) // p)[q > 0].sum())
+    if prob.causal:
+        pairs = q * (k - q) + q * (q + 1) // 2
+    else:
+        pairs = q * k
+    flops = 4 * d * hq * int(pairs.sum())
+    dec = q == 1
+    dec_bytes = (int(k[dec].sum()) * hkv * d * 2 * e + int(dec.sum()) * hkv * d * 2 * e
+                 + int(dec.sum()) * hq * d * e + 4 * int(((k[dec] + p - 1) // p).sum()))
+    return dict(bytes=kv_read + cache_write + q_out + lse + table, flops=flops, tokens=t,
+                decode_kernel_bytes=dec_bytes, prefill_flops=4 * d * hq * int(pairs[q > 1].sum()))
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            m = json.load(f)
+        return dict(hbm=float(m["hbm_gbs"]), tc=float(m["bf16_tflops"]),
+                    tc_sustained=float(m.get("bf16_tflops_sustained", m["bf16_tflops"])),
+                    source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm=6650.0, tc=1590.0, tc_sustained=1400.0, source="fallback")
+
+
+def traffic_for(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's
+    source has not changed since those counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(f"{kernel}/{workload}")
+    except (OSError, ValueError):
+        return None
+    if not rec:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    try:
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    return rec["dram_bytes_per_launch"] if sha == rec["source_sha256"] else None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.path = None
+        try:
+            props = torch.cuda.get_device_properties(device)
+            self.bus = "%08x:%02x:%02x.0" % (getattr(props, "pci_domain_id", 0),
+                                             getattr(props, "pci_bus_id", 0),
+                                             getattr(props, "pci_device_id", 0))
+        except Exception:
+            self.bus = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "50"]
+        if self.bus:
+            cmd += ["-i", self.bus]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        self.proc.wait()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(pw) if pw else None}
+
+
+# ------------------------------------------------------------------ GPU arm
+def device_problem(name: str, causal, device) -> I.Problem:
+    return I.make_workload(name, device=device, causal=causal, poison=False)
+
+
+def time_steps(prob, steps, warmup, flush, stream, profile=False):
+    from ragged_paged_attention_03_b200 import binding
+    out = torch.empty_like(prob.q)
+    lse = torch.empty(prob.q.shape[0], prob.num_q_heads, dtype=torch.float32, device=prob.q.device)
+
+    def call():
+        binding.rpa_forward(prob.q, prob.k_new, prob.v_new, prob.k_cache, prob.v_cache,
+                            prob.page_table, prob.cu_q_lens, prob.kv_lens, prob.distribution,
+                            prob.scale, prob.causal, out, lse, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            flush.add_(1)
+            call()
+        stream.synchronize()
+        if profile:
+            binding.rpa_profile_read()
+            binding.rpa_profile_enable(True)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        for a, b in evs:
+            flush.add_(1)            # 256 MiB write evicts the step's data from L2
+            a.record(stream)
+            call()
+            b.record(stream)
+        stream.synchronize()
+        if profile:
+            binding.rpa_profile_enable(False)
+    kern = binding.rpa_profile_read() if profile else None
+    flags = binding.rpa_device_status(stream)
+    if flags:
+        raise RuntimeError(f"device error flags {flags:#x}")
+    ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    return ms, kern
+
+
+def time_e2e(prob, steps, warmup, flush, stream):
+    """Host buffers in, host buffers out: each step copies this step's Q, new
+    K/V and page table from pinned host memory, runs rpa_forward and copies
+    out and lse back, all inside the timed region."""
+    from ragged_paged_attention_03_b200 import binding
+    h = {k: getattr(prob, k).cpu().pin_memory() for k in ("q", "k_new", "v_new", "page_table")}
+    d = {k: torch.empty_like(getattr(prob, k)) for k in h}
+    out = torch.empty_like(prob.q)
+    lse = torch.empty(prob.q.shape[0], prob.num_q_heads, dtype=torch.float32, device=prob.q.device)
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in h.values())
+    d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * 4
+
+    def call():
+        for k in h:
+            d[k].copy_(h[k], non_blocking=True)
+        binding.rpa_forward(d["q"], d["k_new"], d["v_new"], prob.k_cache, prob.v_cache,
+                            d["page_table"], prob.cu_q_lens, prob.kv_lens, prob.distribution,
+                            prob.scale, prob.causal, out, lse, stream=stream)
+        h_out.copy_(out, non_blocking=True)
+        h_lse.copy_(lse, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            flush.add_(1)
+            call()
+        stream.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        for a, b in evs:
+            flush.add_(1)
+            a.record(stream)
+            call()
+            b.record(stream)
+        stream.synchronize()
+    return float(np.mean([a.elapsed_time(b) for a, b in evs])), h2d, d2h
+
+
+def metric_of(name):
+    if name.startswith("decode"):
+        return "decode HBM GB/s", "GB/s"
+    if name.startswith("prefill"):
+        return "prefill TFLOP/s", "TFLOP/s"
+    if name.startswith("mixed"):
+        return "mixed-batch tokens/s", "tokens/s"
+    return "long-context HBM GB/s", "GB/s"
+
+
+def value_of(name, work, ms, n):
+    metric, unit = metric_of(name)
+    if unit == "GB/s":
+        return n * work["bytes"] / (ms * 1e-3) / 1e9
+    if unit == "TFLOP/s":
+        return n * work["flops"] / (ms * 1e-3) / 1e12
+    return n * work["tokens"] / (ms * 1e-3)
+
+
+def roofline(name, work, kern, pk):
+    """The dominant kernel of the step against its own roofline."""
+    launches = {k: v for k, v in kern.items() if v[0] > 0}
+    top = max(launches, key=lambda k: launches[k][1])
+    n, total_ms = launches[top]
+    avg_s = total_ms / n * 1e-3
+    if top == "prefill":
+        achieved = work["prefill_flops"] / avg_s / 1e12
+        r = {"bound": "tensor", "achieved": achieved, "peak": pk["tc"], "unit": "TFLOP/s",
+             "peak_source": f"{pk['source']} bf16 dense (burst)"}
+    else:
+        b = work["decode_kernel_bytes"] if top == "decode" else work["bytes"]
+        achieved = b / avg_s / 1e9
+        r = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
+             "peak_source": f"{pk['source']} HBM copy"}
+    r["frac"] = r["achieved"] / r["peak"]
+    r["kernel"] = top
+    r["kernel_ms"] = total_ms / n
+    r["traffic"] = traffic_for(top, name)
+    r["kernel_share"] = {k: round(v[1] / sum(x[1] for x in launches.values()), 4)
+                         for k, v in launches.items()}
+    return r
+
+
+# ----------------------------------------------------------- oracle (CPU)
+def oracle_sample(prob_dev: I.Problem, budget_s: float):
+    """Sequences of the workload for a bounded oracle run: decode sequences
+    in order, then prefill sequences, until the estimated fp64 work fills
+    about `budget_s` seconds of the host's cores."""
+    import oracle
+    rate = 0.4e9 * max(1, oracle.num_threads())          # fp64 multiply-adds / s, rough
+    q = prob_dev.q_lens.astype(np.int64)
+    k = prob_dev.kv_lens.astype(np.int64)
+    pairs = q * (k - q) + q * (q + 1) // 2 if prob_dev.causal else q * k
+    cost = 2.0 * pairs * prob_dev.num_q_heads * prob_dev.head_dim
+    order = [s for s in range(prob_dev.num_seqs) if q[s] == 1] + \
+            [s for s in range(prob_dev.num_seqs) if q[s] > 1]
+    pick, acc = [], 0.0
+    for s in order:
+        if pick and acc + cost[s] > rate * budget_s:
+            continue
+        pick.append(s)
+        acc += cost[s]
+    return sorted(pick)
+
+
+def run_oracle_sample(sub: I.Problem):
+    import oracle
+    kc = I.to_storage(sub.k_cache).copy()
+    vc = I.to_storage(sub.v_cache).copy()
+    args = (I.to_storage(sub.q), I.to_storage(sub.k_new), I.to_storage(sub.v_new))
+    t0 = time.perf_counter()
+    oracle.forward(*args, kc, vc, sub.page_table.numpy(), sub.cu_q_lens, sub.kv_lens, sub.scale,
+                   sub.causal, sub.dtype)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(name, prob_dev, budget_s):
+    import oracle
+    seqs = oracle_sample(prob_dev, budget_s)
+    sub = I.sub_problem(prob_dev, seqs)
+    dt = run_oracle_sample(sub)
+    work = algorithmic(sub)
+    metric, unit = metric_of(name)
+    v = value_of(name, work, dt * 1e3, 1)
+    return {"value": v, "unit": unit, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{len(seqs)} of {prob_dev.num_seqs} sequences "
+                      f"({work['tokens']} new tokens, {work['bytes'] / 1e9:.3f} GB, "
+                      f"{work['flops'] / 1e9:.1f} GFLOP), one fp64 oracle pass, {dt:.1f} s"}
+
+
+# ----------------------------------------------------------------- main
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "ours":
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workloads", default="decode_128,prefill_8x2048,prefill_8x2048:noncausal,"
+                                           "mixed_96d_4c,long_d256")
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of oracle work for the cpu_baseline sample")
+    args = ap.parse_args()
+    world, rank, local = dist_setup(args)
+    n = world
+    wl = [w for w in args.workloads.split(",") if w]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        name = wl[0].split(":")[0]
+        prob = I.make_workload(name, device="cpu", poison=False)
+        seqs = oracle_sample(prob, max(1.0, 150.0 / max(1, args.steps + args.warmup)))
+        sub = I.sub_problem(prob, seqs)
+        for _ in range(args.warmup):
+            run_oracle_sample(sub)
+        times = [run_oracle_sample(sub) for _ in range(args.steps)]
+        work = algorithmic(sub)
+        ms = float(np.mean(times)) * 1e3
+        metric, unit = metric_of(name)
+        v = value_of(name, work, ms, 1)
+        import oracle
+        line = {"impl": "reference", "metric": metric, "value": v, "unit": unit, "n_gpus": n,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic",
+                "config": {"workload": WORKLOAD_TEXT[name], "sample_seqs": len(seqs)},
+                "cpu_baseline": {"value": v, "unit": unit, "cores": oracle.num_threads(),
+                                 "kind": "oracle",
+                                 "sample": f"{len(seqs)} of {prob.num_seqs} sequences per step"},
+                "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    from ragged_paged_attention_03_b200 import build
+    if rank == 0 and not os.path.exists(os.path.join(ROOT, "ragged_paged_attention_03_b200",
+                                                     "librpa_b200.so")):
+        build.build()
+    if world > 1:
+        torch.distributed.barrier()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    pk = peaks()
+    clocks = ClockSampler(local)
+    results = []
+    cpu_base = None
+    for i, spec in enumerate(wl):
+        name, _, opt = spec.partition(":")
+        causal = False if opt == "noncausal" else None
+        prob = device_problem(name, causal, dev)
+        work = algorithmic(prob)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        if i == 0:
+            clocks.start()
+        ms, kern = time_steps(prob, args.steps, args.warmup, flush, stream, profile=True)
+        if i == 0:
+            clk = clocks.stop()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            ms = float(t.item())
+            torch.distributed.barrier()
+        e2e_ms, h2d, d2h = time_e2e(prob, max(10, args.steps // 4), 3, flush, stream)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        metric, unit = metric_of(name)
+        line = {"metric": metric, "value": value_of(name, work, ms, n), "unit": unit,
+                "ms_per_step": ms,
+                "workload": name + ("" if prob.causal else " (non-causal)"),
+                "config": {"workload": WORKLOAD_TEXT[name] + ("" if prob.causal else ", non-causal"),
+                           "l2": "flushed between steps (256 MiB write)",
+                           "tokens": work["tokens"], "bytes": work["bytes"],
+                           "flops": work["flops"]},
+                "roofline": roofline(name, work, kern, pk),
+                "e2e": {"value": value_of(name, work, e2e_ms, n), "unit": unit,
+                        "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h},
+                "gpu_launches": int(sum(v[0] for v in kern.values()))}
+        if rank == 0 and i == 0 and world == 1:
+            cpu_base = cpu_baseline(name, prob, args.cpu_budget)
+        results.append(line)
+        del prob
+        torch.cuda.empty_cache()
+    if rank == 0:
+        head = results[0]
+        out = {"metric": head["metric"], "value": head["value"], "unit": head["unit"],
+               "n_gpus": n, "steps": args.steps, "warmup": args.warmup,
+               "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+               "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+               "config": {**head["config"], "parallelism": f"replicas x{n}" if n > 1 else "1 GPU"},
+               "roofline": head["roofline"], "e2e": head["e2e"],
+               "gpu_launches": head["gpu_launches"], "clocks": clk,
+               "cpu_baseline": cpu_base, "also": results[1:]}
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

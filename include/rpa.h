@@ -1,0 +1,205 @@
+/*
+ * rpa.h -- C ABI of librpa_b200.so: ragged paged attention on NVIDIA B200
+ * (sm_100a).
+ *
+ * The operation ("Ragged Paged Attention: A High-Performance and Flexible LLM
+ * Inference Kernel for TPU", arXiv 2604.15464, abstract): one attention pass
+ * over a ragged batch whose sequences may be decoding (one new token),
+ * prefilling (every token new) or both (new tokens after a cached context),
+ * where each sequence's keys and values live in fixed-size pages of a shared
+ * pool addressed through a per-sequence page table (RPA talk summary,
+ * rocketrecap.com, glossary "PagedAttention"), and where the new tokens' K/V
+ * are written into their cache pages by the same kernels that attend over
+ * them (talk summary 00:06:36).  Attention is exact softmax attention
+ * (glossary "FlashAttention"); the result does not depend on how the batch
+ * is split across kernels.
+ *
+ * Notation: S sequences; sequence s has q_len[s] = cu_q_lens[s+1] -
+ * cu_q_lens[s] new tokens and kv_len[s] >= q_len[s] tokens in total, so its
+ * first c[s] = kv_len[s] - q_len[s] tokens are already cached.  T =
+ * cu_q_lens[S] new tokens in all.  Hq query heads, Hkv KV heads, G = Hq/Hkv;
+ * query head h reads KV head h / G.  D = head_dim, P = page_size.
+ *
+ * All functions are thread-safe, never throw, never abort and never free
+ * memory they did not allocate.
+ */
+#ifndef RPA_H
+#define RPA_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RPA_API __attribute__((visibility("default")))
+#else
+#define RPA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element type of q, k_new, v_new, the caches and out (all the same). */
+typedef enum { RPA_F32 = 0, RPA_BF16 = 1 } rpa_dtype;
+
+/* Return codes. */
+enum {
+  RPA_OK = 0,
+  RPA_ERR_INVALID_ARG = 1,   /* null pointer where one is required, bad dims */
+  RPA_ERR_UNSUPPORTED = 2,   /* head_dim not in {64,128,256}; page_size not a
+                                power of two in [8,256]; Hq % Hkv != 0; G > 16 */
+  RPA_ERR_LENGTHS = 3,       /* cu_q_lens not starting at 0 / decreasing;
+                                kv_len < q_len; more pages than
+                                max_pages_per_seq; T != total_q_tokens */
+  RPA_ERR_DISTRIBUTION = 4,  /* distribution given and inconsistent */
+  RPA_ERR_OOM = 5,           /* library workspace could not be allocated */
+  RPA_ERR_CUDA = 6           /* a CUDA call or kernel launch failed */
+};
+
+/* Bits of the device error word read by rpa_device_status(). */
+#define RPA_DEV_BAD_PAGE 0x1u /* a page-table entry outside [0, num_pages)
+                                 was met; that page was read as zeros and
+                                 nothing was written to it */
+#define RPA_DEV_TIMEOUT 0x2u  /* a bounded wait on a shared-memory barrier ran
+                                 out; the CTA stopped early, outputs of that
+                                 CTA are incomplete */
+
+/* Problem geometry. */
+typedef struct {
+  int32_t num_q_heads;       /* Hq */
+  int32_t num_kv_heads;      /* Hkv, divides Hq */
+  int32_t head_dim;          /* D: 64, 128 or 256 */
+  int32_t page_size;         /* P: power of two, 8..256 */
+  int32_t num_pages;         /* physical pages in each cache */
+  int32_t max_pages_per_seq; /* row length of page_table */
+  int32_t total_q_tokens;    /* T, must equal cu_q_lens[num_seqs] */
+  int32_t dtype;             /* rpa_dtype */
+} rpa_dims;
+
+/*
+ * rpa_forward -- one ragged paged attention pass.
+ *
+ * Device buffers (row-major, contiguous, all of dims->dtype unless noted):
+ *   q        [T, Hq, D]       read
+ *   k_new    [T, Hkv, D]      read: K of the new tokens, in token order
+ *   v_new    [T, Hkv, D]      read
+ *   k_cache  [num_pages, P, Hkv, D]  read and written in place
+ *   v_cache  [num_pages, P, Hkv, D]  read and written in place
+ *   page_table [num_seqs, max_pages_per_seq] int32: logical page j of
+ *            sequence s is physical page page_table[s][j]; only the first
+ *            ceil(kv_len[s] / P) entries of a row are read
+ *   out      [T, Hq, D]       written for every row
+ *   lse      [T, Hq] float32  written for every row, or NULL
+ * Host buffers:
+ *   cu_q_lens [num_seqs + 1] int32, cu_q_lens[0] = 0, non-decreasing
+ *   kv_lens   [num_seqs] int32, kv_len[s] >= q_len[s]
+ *   distribution [3] int32 or NULL: cumulative counts {d, p, S}.  Sequences
+ *            [0, d) are decode (q_len <= 1), [d, p) fresh prefill
+ *            (q_len == kv_len), [p, S) mixed / chunked prefill (any q_len <=
+ *            kv_len).  This is the pages' distribution-aware split into
+ *            decode, prefill and mixed work (arXiv 2604.15464, abstract,
+ *            technique 3).  NULL: the library classifies each sequence
+ *            itself and sequence order does not matter.  It only chooses
+ *            kernels; results never depend on it.
+ *
+ * Semantics (exact attention; talk summary 00:06:36 for the order):
+ *   1. for every s and i < q_len[s], K/V of new token cu_q_lens[s] + i are
+ *      copied bit for bit into slot (c[s] + i) % P of physical page
+ *      page_table[s][(c[s] + i) / P] of k_cache / v_cache;
+ *   2. query row t = cu_q_lens[s] + i, head h attends over positions
+ *      j < kv_len[s] of the updated cache with KV head h / G, restricted to
+ *      j <= c[s] + i when causal != 0 (the mask is aligned to the end of the
+ *      sequence): out = sum_j softmax_j(scale * q.k_j) v_j, accumulated in
+ *      fp32 and rounded to nearest-even into dtype;
+ *      lse = ln sum_j exp(scale * q.k_j) over the same positions (fp32).
+ *   Cache slots other than those of step 1 are never written; slots past
+ *   kv_len and unused pages are never read (they may hold NaN).
+ *
+ * Ownership and aliasing: the caller owns every buffer.  out and lse must
+ * not overlap any input.  Pages written by one call must not be shared by
+ * two sequences of that call.  The library keeps a per-device workspace
+ * (descriptor buffers, split-KV partials, the error word) that it grows on
+ * demand and frees at process exit.
+ *
+ * stream: a cudaStream_t (NULL = legacy default stream).  The call is
+ * asynchronous: it validates and plans on the host, queues one small
+ * host-to-device copy of the plan and the kernels on `stream`, and returns.
+ * num_seqs == 0 or T == 0 with no kv work is a successful no-op.
+ *
+ * Returns RPA_OK or an RPA_ERR_* code; on an error nothing was queued and no
+ * buffer was touched.  Device-side conditions are reported through
+ * rpa_device_status().
+ */
+RPA_API int rpa_forward(const void *q, const void *k_new, const void *v_new,
+                void *k_cache, void *v_cache, const int32_t *page_table,
+                const int32_t *cu_q_lens, const int32_t *kv_lens,
+                int32_t num_seqs, const int32_t *distribution, float scale,
+                int32_t causal, void *out, float *lse, const rpa_dims *dims,
+                void *stream);
+
+/*
+ * rpa_device_status -- synchronise `stream`, then read and clear the current
+ * device's error word (RPA_DEV_* bits, 0 when nothing happened) into *flags.
+ * Returns RPA_OK, or RPA_ERR_CUDA if the synchronisation reported an error.
+ */
+RPA_API int rpa_device_status(void *stream, uint32_t *flags);
+
+/* Static, human-readable name of a return code. */
+RPA_API const char *rpa_status_string(int status);
+
+/* What the host planner made of a batch (host only, no GPU needed). */
+typedef struct {
+  int32_t num_decode;        /* sequences run by the decode kernel */
+  int32_t num_prefill;       /* sequences run by the prefill kernel */
+  int32_t num_generic;       /* sequences run by the generic kernel */
+  int32_t num_empty;         /* q_len == 0 sequences */
+  int32_t decode_items;      /* (sequence, kv chunk) work items, per KV head */
+  int32_t decode_max_splits; /* most chunks any one decode sequence got */
+  int32_t combine_rows;      /* decode sequences that need the LSE combine */
+  int32_t prefill_tiles;     /* (sequence, query tile) work items, per Q head */
+  int64_t plan_bytes;        /* bytes of the plan copied to the device */
+} rpa_plan_info;
+
+/*
+ * rpa_plan -- run validation and the host planner exactly as rpa_forward
+ * would for these lengths and dims, without touching any device.  Returns
+ * the same RPA_ERR_* codes rpa_forward would; fills *info on RPA_OK.
+ */
+RPA_API int rpa_plan(const int32_t *cu_q_lens, const int32_t *kv_lens,
+             int32_t num_seqs, const int32_t *distribution,
+             const rpa_dims *dims, rpa_plan_info *info);
+
+/* Planner knobs (process-wide).  Each returns the previous value. */
+enum {
+  RPA_OPT_DECODE_CHUNK_BLOCKS = 0, /* 16-token blocks per decode work item
+                                      (default 64; <= 0 restores it) */
+  RPA_OPT_FORCE_GENERIC = 1,       /* 1: run every sequence on the generic
+                                      kernel (default 0) */
+  RPA_OPT_DISABLE_PREFILL_TC = 2   /* 1: prefill sequences use the generic
+                                      kernel instead of tensor cores */
+};
+RPA_API int64_t rpa_set_option(int32_t option, int64_t value);
+
+/* Kernel classes reported by rpa_profile_read(). */
+enum { RPA_KERNEL_GENERIC = 0, RPA_KERNEL_DECODE = 1, RPA_KERNEL_COMBINE = 2,
+       RPA_KERNEL_PREFILL = 3, RPA_KERNEL_CLASSES = 4 };
+
+/*
+ * rpa_profile_enable -- tracing switch (process-wide, default off).  While
+ * on, every kernel launch of rpa_forward is bracketed by two CUDA events on
+ * the launching stream.  Returns the previous setting.
+ */
+RPA_API int32_t rpa_profile_enable(int32_t on);
+
+/*
+ * rpa_profile_read -- wait for every traced launch, add up their device
+ * durations per kernel class and forget them.  ms[RPA_KERNEL_CLASSES]
+ * receives milliseconds, launches[RPA_KERNEL_CLASSES] launch counts (either
+ * may be NULL).  Returns RPA_OK or RPA_ERR_CUDA.
+ */
+RPA_API int rpa_profile_read(double *ms, int64_t *launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RPA_H */

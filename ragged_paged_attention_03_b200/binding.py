@@ -1,0 +1,183 @@
+"""ctypes binding of include/rpa.h -- argument marshalling only.
+
+Every function here has the name of the C entry point it calls and does no
+computation of its own: it checks types and shapes, turns torch tensors into
+device pointers and numpy arrays into host pointers, and raises on a non-zero
+return code.  The library must have been built in-tree
+(``python -m ragged_paged_attention_03_b200.build``); importing this module
+without it raises, so nothing can silently run without the CUDA path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librpa_b200.so")
+
+RPA_F32, RPA_BF16 = 0, 1
+RPA_OK = 0
+RPA_DEV_BAD_PAGE = 0x1
+RPA_DEV_TIMEOUT = 0x2
+RPA_OPT_DECODE_CHUNK_BLOCKS = 0
+RPA_OPT_FORCE_GENERIC = 1
+RPA_OPT_DISABLE_PREFILL_TC = 2
+
+
+class rpa_dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "num_q_heads", "num_kv_heads", "head_dim", "page_size", "num_pages",
+        "max_pages_per_seq", "total_q_tokens", "dtype")]
+
+
+class rpa_plan_info(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "num_decode", "num_prefill", "num_generic", "num_empty", "decode_items",
+        "decode_max_splits", "combine_rows", "prefill_tiles")] + [("plan_bytes", ctypes.c_int64)]
+
+
+class RpaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {rpa_status_string(code)} (code {code})")
+        self.code = code
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with "
+                      "`python -m ragged_paged_attention_03_b200.build`")
+_lib = ctypes.CDLL(LIB_PATH)
+_P = ctypes.c_void_p
+_i32 = ctypes.c_int32
+_lib.rpa_forward.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _i32, _P, ctypes.c_float, _i32, _P,
+                             _P, ctypes.POINTER(rpa_dims), _P]
+_lib.rpa_forward.restype = ctypes.c_int
+_lib.rpa_device_status.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32)]
+_lib.rpa_device_status.restype = ctypes.c_int
+_lib.rpa_status_string.argtypes = [ctypes.c_int]
+_lib.rpa_status_string.restype = ctypes.c_char_p
+_lib.rpa_plan.argtypes = [_P, _P, _i32, _P, ctypes.POINTER(rpa_dims), ctypes.POINTER(rpa_plan_info)]
+_lib.rpa_plan.restype = ctypes.c_int
+_lib.rpa_set_option.argtypes = [_i32, ctypes.c_int64]
+_lib.rpa_set_option.restype = ctypes.c_int64
+_lib.rpa_profile_enable.argtypes = [_i32]
+_lib.rpa_profile_enable.restype = ctypes.c_int32
+_lib.rpa_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
+_lib.rpa_profile_read.restype = ctypes.c_int
+KERNEL_CLASSES = ("generic", "decode", "combine", "prefill")
+
+
+def library() -> ctypes.CDLL:
+    return _lib
+
+
+def rpa_status_string(code: int) -> str:
+    return _lib.rpa_status_string(int(code)).decode()
+
+
+def rpa_set_option(option: int, value: int) -> int:
+    return int(_lib.rpa_set_option(int(option), int(value)))
+
+
+def _host_i32(a) -> Optional[np.ndarray]:
+    if a is None:
+        return None
+    if isinstance(a, torch.Tensor):
+        a = a.cpu().numpy()
+    return np.ascontiguousarray(a, dtype=np.int32)
+
+
+def _hp(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(_P)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return RPA_F32
+    if t.dtype == torch.bfloat16:
+        return RPA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def make_dims(q: torch.Tensor, k_cache: torch.Tensor, page_table: torch.Tensor) -> rpa_dims:
+    num_pages, page_size, hkv, d = k_cache.shape
+    return rpa_dims(num_q_heads=q.shape[1], num_kv_heads=hkv, head_dim=d, page_size=page_size,
+                    num_pages=num_pages, max_pages_per_seq=page_table.shape[1],
+                    total_q_tokens=q.shape[0], dtype=_dtype_code(q))
+
+
+def rpa_plan(cu_q_lens, kv_lens, distribution, dims: rpa_dims) -> rpa_plan_info:
+    cu, kv, dist = _host_i32(cu_q_lens), _host_i32(kv_lens), _host_i32(distribution)
+    info = rpa_plan_info()
+    rc = _lib.rpa_plan(_hp(cu), _hp(kv), len(kv), _hp(dist), ctypes.byref(dims), ctypes.byref(info))
+    if rc != RPA_OK:
+        raise RpaError(rc, "rpa_plan")
+    return info
+
+
+def _dev(t: Optional[torch.Tensor], name: str, dtype=None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def rpa_forward(q, k_new, v_new, k_cache, v_cache, page_table, cu_q_lens, kv_lens, distribution,
+                scale: float, causal: bool, out, lse=None, stream=None) -> None:
+    """Calls rpa_forward on `stream` (default: torch's current stream).
+
+    Device tensors: q [T,Hq,D], k_new/v_new [T,Hkv,D], k_cache/v_cache
+    [pages,P,Hkv,D], page_table [S,max_pages] int32, out [T,Hq,D], lse [T,Hq]
+    float32 or None.  Host arrays: cu_q_lens [S+1], kv_lens [S], distribution
+    [3] or None (int32)."""
+    dt = q.dtype
+    for name, t in (("k_new", k_new), ("v_new", v_new), ("k_cache", k_cache),
+                    ("v_cache", v_cache), ("out", out)):
+        if t.dtype != dt:
+            raise TypeError(f"{name} dtype {t.dtype} != q dtype {dt}")
+    cu, kv, dist = _host_i32(cu_q_lens), _host_i32(kv_lens), _host_i32(distribution)
+    dims = make_dims(q, k_cache, page_table)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    sptr = ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+    rc = _lib.rpa_forward(_dev(q, "q"), _dev(k_new, "k_new"), _dev(v_new, "v_new"),
+                          _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                          _dev(page_table, "page_table", torch.int32), _hp(cu), _hp(kv), len(kv),
+                          _hp(dist), float(scale), int(bool(causal)), _dev(out, "out"),
+                          _dev(lse, "lse", torch.float32), ctypes.byref(dims), sptr)
+    if rc != RPA_OK:
+        raise RpaError(rc, "rpa_forward")
+
+
+def rpa_device_status(stream=None) -> int:
+    """Synchronises `stream` and returns (and clears) the device error bits."""
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    sptr = ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+    flags = ctypes.c_uint32(0)
+    rc = _lib.rpa_device_status(sptr, ctypes.byref(flags))
+    if rc != RPA_OK:
+        raise RpaError(rc, "rpa_device_status")
+    return int(flags.value)
+
+
+def rpa_profile_enable(on: bool) -> bool:
+    return bool(_lib.rpa_profile_enable(int(bool(on))))
+
+
+def rpa_profile_read() -> dict:
+    """{kernel class: (launches, total ms)} since the last read."""
+    ms = (ctypes.c_double * 4)()
+    n = (ctypes.c_int64 * 4)()
+    rc = _lib.rpa_profile_read(ms, n)
+    if rc != RPA_OK:
+        raise RpaError(rc, "rpa_profile_read")
+    return {k: (int(n[i]), float(ms[i])) for i, k in enumerate(KERNEL_CLASSES)}

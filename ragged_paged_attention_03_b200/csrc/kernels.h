@@ -1,0 +1,47 @@
+// kernels.h -- launch interface between the host planner and the kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "plan.h"
+
+namespace rpa {
+
+// Device pointers and geometry shared by every kernel of one call.
+struct Problem {
+  const void *q;
+  const void *k_new;
+  const void *v_new;
+  void *k_cache;
+  void *v_cache;
+  const int32_t *page_table;
+  void *out;
+  float *lse;          // may be null
+  uint32_t *err;       // device error word (RPA_DEV_* bits)
+  int32_t hq, hkv, d, p, num_pages, max_pages, dtype, causal;
+  float scale;
+};
+
+// Generic SIMT kernel: any dtype, any q_len, one warp per (row, query head).
+cudaError_t launch_generic(const Problem &pb, const GenericSeq *seqs,
+                           int n_seqs, int n_rows, cudaStream_t stream);
+
+// Decode kernel (bf16): one CTA per (work item, KV head).
+// partial_o: [n_partials, Hkv, G, D] fp32; partial_lse: [n_partials, Hkv, G].
+cudaError_t launch_decode(const Problem &pb, const DecodeItem *items,
+                          int n_items, float *partial_o, float *partial_lse,
+                          cudaStream_t stream);
+
+// Split-KV combine: one warp per (combine item, query head).
+cudaError_t launch_combine(const Problem &pb, const CombineItem *items,
+                           int n_items, const float *partial_o,
+                           const float *partial_lse, cudaStream_t stream);
+
+// Prefill / chunked-prefill kernel (bf16, tcgen05): one CTA per (tile, query head).
+cudaError_t launch_prefill(const Problem &pb, const PrefillTile *tiles,
+                           int n_tiles, cudaStream_t stream);
+
+// Rows per prefill tile (query tokens per CTA tile).
+constexpr int kPrefillTileRows = 128;
+
+}  // namespace rpa

@@ -1,0 +1,500 @@
+// rpa_api.cu -- the C ABI of include/rpa.h: validation, the host planner,
+// the per-device workspace and the kernel launches of one rpa_forward call.
+//
+// The planner is the B200 counterpart of the distribution-aware
+// specialisation in "Ragged Paged Attention" (arXiv 2604.15464), abstract,
+// technique 3: each sequence is routed to the kernel specialised for its
+// shape (decode: one new token; prefill / chunked prefill: many), and the
+// per-kernel work lists are built on the host, uploaded with one copy and
+// consumed by the kernels.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+#include <atomic>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "kernels.h"
+#include "plan.h"
+#include "rpa.h"
+
+namespace rpa {
+namespace {
+
+std::atomic<int64_t> g_opt_decode_chunk{0};
+std::atomic<int64_t> g_opt_force_generic{0};
+std::atomic<int64_t> g_opt_disable_prefill_tc{0};
+
+constexpr int kDefaultDecodeChunkBlocks = 64;
+constexpr bool kHaveDecodeKernel = false;
+constexpr bool kHavePrefillKernel = false;
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+int validate_dims(const rpa_dims *d) {
+  if (d == nullptr) return RPA_ERR_INVALID_ARG;
+  if (d->num_q_heads <= 0 || d->num_kv_heads <= 0 || d->num_pages <= 0 ||
+      d->max_pages_per_seq <= 0 || d->total_q_tokens < 0 ||
+      (d->dtype != RPA_F32 && d->dtype != RPA_BF16))
+    return RPA_ERR_INVALID_ARG;
+  if (d->head_dim != 64 && d->head_dim != 128 && d->head_dim != 256) return RPA_ERR_UNSUPPORTED;
+  if (!is_pow2(d->page_size) || d->page_size < 8 || d->page_size > 256) return RPA_ERR_UNSUPPORTED;
+  if (d->num_q_heads % d->num_kv_heads != 0) return RPA_ERR_UNSUPPORTED;
+  if (d->num_q_heads / d->num_kv_heads > 16) return RPA_ERR_UNSUPPORTED;
+  return RPA_OK;
+}
+
+int validate_lengths(const int32_t *cu, const int32_t *kv, int32_t n, const rpa_dims *d) {
+  if (n < 0) return RPA_ERR_INVALID_ARG;
+  if (n == 0) return d->total_q_tokens == 0 ? RPA_OK : RPA_ERR_LENGTHS;
+  if (cu == nullptr || kv == nullptr) return RPA_ERR_INVALID_ARG;
+  if (cu[0] != 0) return RPA_ERR_LENGTHS;
+  const int64_t cap = (int64_t)d->max_pages_per_seq * d->page_size;
+  for (int32_t s = 0; s < n; ++s) {
+    int64_t ql = (int64_t)cu[s + 1] - cu[s];
+    if (ql < 0 || kv[s] < ql || (int64_t)kv[s] > cap) return RPA_ERR_LENGTHS;
+  }
+  if (cu[n] != d->total_q_tokens) return RPA_ERR_LENGTHS;
+  return RPA_OK;
+}
+
+int validate_distribution(const int32_t *dist, const int32_t *cu, const int32_t *kv, int32_t n) {
+  if (dist == nullptr) return RPA_OK;
+  const int32_t dd = dist[0], pp = dist[1], ss = dist[2];
+  if (dd < 0 || dd > pp || pp > ss || ss != n) return RPA_ERR_DISTRIBUTION;
+  for (int32_t s = 0; s < n; ++s) {
+    int32_t ql = cu[s + 1] - cu[s];
+    if (s < dd && ql > 1) return RPA_ERR_DISTRIBUTION;
+    if (s >= dd && s < pp && ql != kv[s]) return RPA_ERR_DISTRIBUTION;
+  }
+  return RPA_OK;
+}
+
+enum Route { kEmpty, kGeneric, kDecode, kPrefill };
+
+// Kernel choice for one sequence.  With a distribution the ranges decide the
+// specialisation directly; without one the lengths do.  Both give the same
+// answer for consistent input, and neither affects the result.
+Route route_of(int32_t ql, int32_t kvl, int dtype, int cls) {
+  (void)kvl;
+  if (ql == 0) return kEmpty;
+  if (dtype != RPA_BF16 || g_opt_force_generic.load()) return kGeneric;
+  const bool decode = cls >= 0 ? (cls == 0 || ql == 1) : ql == 1;
+  if (decode) return kHaveDecodeKernel ? kDecode : kGeneric;
+  if (!kHavePrefillKernel || g_opt_disable_prefill_tc.load()) return kGeneric;
+  return kPrefill;
+}
+
+struct HostPlan {
+  std::vector<GenericSeq> generic;
+  std::vector<DecodeItem> decode;
+  std::vector<CombineItem> combine;
+  std::vector<PrefillTile> prefill;
+  int32_t n_generic_rows = 0;
+  int32_t n_partials = 0;
+  int32_t decode_max_splits = 0;
+  int32_t num_decode = 0, num_prefill = 0, num_generic = 0, num_empty = 0;
+  PlanLayout layout{};
+};
+
+void build_plan(const int32_t *cu, const int32_t *kv, int32_t n, const int32_t *dist,
+                const rpa_dims *d, HostPlan &hp) {
+  int64_t chunk = g_opt_decode_chunk.load();
+  if (chunk <= 0) chunk = kDefaultDecodeChunkBlocks;
+  for (int32_t s = 0; s < n; ++s) {
+    const int32_t ql = cu[s + 1] - cu[s];
+    const int32_t kvl = kv[s];
+    int cls = -1;
+    if (dist) cls = s < dist[0] ? 0 : (s < dist[1] ? 1 : 2);
+    switch (route_of(ql, kvl, d->dtype, cls)) {
+      case kEmpty:
+        ++hp.num_empty;
+        break;
+      case kGeneric: {
+        GenericSeq g{};
+        g.seq = s;
+        g.q_start = cu[s];
+        g.q_len = ql;
+        g.kv_len = kvl;
+        g.row_prefix = hp.n_generic_rows;
+        hp.n_generic_rows += ql;
+        hp.generic.push_back(g);
+        ++hp.num_generic;
+        break;
+      }
+      case kDecode: {
+        ++hp.num_decode;
+        const int32_t nblk = (kvl + kDecodeBlock - 1) / kDecodeBlock;
+        const int32_t nsplit = (int32_t)((nblk + chunk - 1) / chunk);
+        const int32_t per = (nblk + nsplit - 1) / nsplit;
+        hp.decode_max_splits = std::max(hp.decode_max_splits, nsplit);
+        const int32_t first_partial = hp.n_partials;
+        int32_t made = 0;
+        for (int32_t b = 0; b < nblk; b += per) {
+          DecodeItem it{};
+          it.seq = s;
+          it.token = cu[s];
+          it.kv_len = kvl;
+          it.blk_begin = b;
+          it.blk_end = std::min(nblk, b + per);
+          it.owns_new = it.blk_end == nblk ? 1 : 0;
+          it.partial = nsplit > 1 ? hp.n_partials++ : -1;
+          hp.decode.push_back(it);
+          ++made;
+        }
+        if (made > 1) {
+          CombineItem c{};
+          c.token = cu[s];
+          c.first_partial = first_partial;
+          c.nsplit = made;
+          hp.combine.push_back(c);
+        }
+        break;
+      }
+      case kPrefill: {
+        ++hp.num_prefill;
+        for (int32_t r = 0; r < ql; r += kPrefillTileRows) {
+          PrefillTile t{};
+          t.seq = s;
+          t.q_start = cu[s];
+          t.q_len = ql;
+          t.kv_len = kvl;
+          t.tile_row = r;
+          t.rows = std::min(kPrefillTileRows, ql - r);
+          hp.prefill.push_back(t);
+        }
+        break;
+      }
+    }
+  }
+  // Heaviest prefill tiles first: with a causal mask a tile's key range ends
+  // at its last row, so later tiles of a sequence carry more work.
+  std::stable_sort(hp.prefill.begin(), hp.prefill.end(),
+                   [](const PrefillTile &a, const PrefillTile &b) {
+                     int64_t wa = (int64_t)(a.kv_len - a.q_len + a.tile_row + a.rows);
+                     int64_t wb = (int64_t)(b.kv_len - b.q_len + b.tile_row + b.rows);
+                     return wa > wb;
+                   });
+  PlanLayout &L = hp.layout;
+  int64_t off = 0;
+  L.generic_off = off;
+  L.n_generic_seqs = (int64_t)hp.generic.size();
+  L.n_generic_rows = hp.n_generic_rows;
+  off += L.n_generic_seqs * (int64_t)(sizeof(GenericSeq) / 4);
+  L.decode_off = off;
+  L.n_decode_items = (int64_t)hp.decode.size();
+  off += L.n_decode_items * (int64_t)(sizeof(DecodeItem) / 4);
+  L.combine_off = off;
+  L.n_combine = (int64_t)hp.combine.size();
+  off += L.n_combine * (int64_t)(sizeof(CombineItem) / 4);
+  L.prefill_off = off;
+  L.n_prefill_tiles = (int64_t)hp.prefill.size();
+  off += L.n_prefill_tiles * (int64_t)(sizeof(PrefillTile) / 4);
+  L.n_partials = hp.n_partials;
+  L.total_words = off;
+}
+
+void serialize(const HostPlan &hp, int32_t *dst) {
+  const PlanLayout &L = hp.layout;
+  if (!hp.generic.empty())
+    memcpy(dst + L.generic_off, hp.generic.data(), hp.generic.size() * sizeof(GenericSeq));
+  if (!hp.decode.empty())
+    memcpy(dst + L.decode_off, hp.decode.data(), hp.decode.size() * sizeof(DecodeItem));
+  if (!hp.combine.empty())
+    memcpy(dst + L.combine_off, hp.combine.data(), hp.combine.size() * sizeof(CombineItem));
+  if (!hp.prefill.empty())
+    memcpy(dst + L.prefill_off, hp.prefill.data(), hp.prefill.size() * sizeof(PrefillTile));
+}
+
+// ---------------------------------------------------------------- workspace
+//
+// Per device: a ring of slots, each with a pinned host staging buffer, a
+// device plan buffer, a split-KV partial buffer and an event recorded after
+// the slot's last kernel.  A slot is reused only once its event has fired,
+// so calls on different streams never overwrite a plan or partials that a
+// queued kernel still reads.
+constexpr int kSlots = 4;
+constexpr int kMaxDevices = 64;
+
+struct Slot {
+  int32_t *host = nullptr;
+  int32_t *dev = nullptr;
+  int64_t words = 0;
+  float *partial = nullptr;  // o then lse
+  int64_t partial_floats = 0;
+  cudaEvent_t done = nullptr;
+  bool pending = false;
+};
+
+struct DeviceWs {
+  std::mutex mu;
+  bool init = false;
+  uint32_t *err = nullptr;
+  Slot slots[kSlots];
+  int next = 0;
+};
+
+DeviceWs g_ws[kMaxDevices];
+
+int ensure_init(DeviceWs &ws) {
+  if (ws.init) return RPA_OK;
+  if (cudaMalloc(&ws.err, sizeof(uint32_t)) != cudaSuccess) return RPA_ERR_OOM;
+  if (cudaMemset(ws.err, 0, sizeof(uint32_t)) != cudaSuccess) return RPA_ERR_CUDA;
+  for (auto &s : ws.slots)
+    if (cudaEventCreateWithFlags(&s.done, cudaEventDisableTiming) != cudaSuccess) return RPA_ERR_CUDA;
+  ws.init = true;
+  return RPA_OK;
+}
+
+int grow_slot(Slot &s, int64_t words, int64_t partial_floats) {
+  if (s.pending) {
+    if (cudaEventSynchronize(s.done) != cudaSuccess) return RPA_ERR_CUDA;
+    s.pending = false;
+  }
+  if (words > s.words) {
+    int64_t w = std::max<int64_t>(words, 2 * s.words);
+    w = std::max<int64_t>(w, 4096);
+    if (s.host) cudaFreeHost(s.host);
+    if (s.dev) cudaFree(s.dev);
+    s.host = nullptr;
+    s.dev = nullptr;
+    s.words = 0;
+    if (cudaMallocHost(&s.host, w * sizeof(int32_t)) != cudaSuccess) return RPA_ERR_OOM;
+    if (cudaMalloc(&s.dev, w * sizeof(int32_t)) != cudaSuccess) return RPA_ERR_OOM;
+    s.words = w;
+  }
+  if (partial_floats > s.partial_floats) {
+    int64_t f = std::max<int64_t>(partial_floats, s.partial_floats + s.partial_floats / 2);
+    if (s.partial) cudaFree(s.partial);
+    s.partial = nullptr;
+    s.partial_floats = 0;
+    if (cudaMalloc(&s.partial, f * sizeof(float)) != cudaSuccess) return RPA_ERR_OOM;
+    s.partial_floats = f;
+  }
+  return RPA_OK;
+}
+
+int plan_checked(const int32_t *cu, const int32_t *kv, int32_t n, const int32_t *dist,
+                 const rpa_dims *d, HostPlan &hp) {
+  int rc = validate_dims(d);
+  if (rc) return rc;
+  rc = validate_lengths(cu, kv, n, d);
+  if (rc) return rc;
+  if (n > 0) rc = validate_distribution(dist, cu, kv, n);
+  if (rc) return rc;
+  build_plan(cu, kv, n, dist, d, hp);
+  return RPA_OK;
+}
+
+
+// ---------------------------------------------------------------- tracing
+std::atomic<int32_t> g_profile_on{0};
+std::mutex g_profile_mu;
+struct Traced {
+  int kind;
+  cudaEvent_t a, b;
+};
+std::vector<Traced> g_traced;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t take_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Runs `launch` on `stream`, bracketed by events when tracing is on.
+template <typename F>
+cudaError_t traced(int kind, cudaStream_t stream, F &&launch) {
+  if (!g_profile_on.load()) return launch();
+  std::lock_guard<std::mutex> lock(g_profile_mu);
+  Traced t{kind, take_event(), take_event()};
+  if (!t.a || !t.b) return launch();
+  cudaEventRecord(t.a, stream);
+  cudaError_t e = launch();
+  cudaEventRecord(t.b, stream);
+  g_traced.push_back(t);
+  return e;
+}
+
+}  // namespace
+}  // namespace rpa
+
+using namespace rpa;
+
+extern "C" RPA_API const char *rpa_status_string(int status) {
+  switch (status) {
+    case RPA_OK: return "ok";
+    case RPA_ERR_INVALID_ARG: return "invalid argument";
+    case RPA_ERR_UNSUPPORTED: return "unsupported geometry";
+    case RPA_ERR_LENGTHS: return "invalid sequence lengths";
+    case RPA_ERR_DISTRIBUTION: return "distribution inconsistent with lengths";
+    case RPA_ERR_OOM: return "workspace allocation failed";
+    case RPA_ERR_CUDA: return "CUDA error";
+    default: return "unknown status";
+  }
+}
+
+extern "C" RPA_API int64_t rpa_set_option(int32_t option, int64_t value) {
+  switch (option) {
+    case RPA_OPT_DECODE_CHUNK_BLOCKS: return g_opt_decode_chunk.exchange(value);
+    case RPA_OPT_FORCE_GENERIC: return g_opt_force_generic.exchange(value);
+    case RPA_OPT_DISABLE_PREFILL_TC: return g_opt_disable_prefill_tc.exchange(value);
+    default: return -1;
+  }
+}
+
+extern "C" RPA_API int rpa_plan(const int32_t *cu_q_lens, const int32_t *kv_lens, int32_t num_seqs,
+                        const int32_t *distribution, const rpa_dims *dims, rpa_plan_info *info) {
+  if (info == nullptr) return RPA_ERR_INVALID_ARG;
+  try {
+    HostPlan hp;
+    int rc = plan_checked(cu_q_lens, kv_lens, num_seqs, distribution, dims, hp);
+    if (rc) return rc;
+    info->num_decode = hp.num_decode;
+    info->num_prefill = hp.num_prefill;
+    info->num_generic = hp.num_generic;
+    info->num_empty = hp.num_empty;
+    info->decode_items = (int32_t)hp.decode.size();
+    info->decode_max_splits = hp.decode_max_splits;
+    info->combine_rows = (int32_t)hp.combine.size();
+    info->prefill_tiles = (int32_t)hp.prefill.size();
+    info->plan_bytes = hp.layout.total_words * 4;
+    return RPA_OK;
+  } catch (const std::bad_alloc &) {
+    return RPA_ERR_OOM;
+  }
+}
+
+extern "C" RPA_API int rpa_forward(const void *q, const void *k_new, const void *v_new, void *k_cache,
+                           void *v_cache, const int32_t *page_table, const int32_t *cu_q_lens,
+                           const int32_t *kv_lens, int32_t num_seqs, const int32_t *distribution,
+                           float scale, int32_t causal, void *out, float *lse,
+                           const rpa_dims *dims, void *stream_ptr) {
+  cudaStream_t stream = (cudaStream_t)stream_ptr;
+  try {
+    HostPlan hp;
+    int rc = plan_checked(cu_q_lens, kv_lens, num_seqs, distribution, dims, hp);
+    if (rc) return rc;
+    const int32_t T = dims->total_q_tokens;
+    if (num_seqs == 0 || T == 0) return RPA_OK;  // no new tokens: nothing to write or attend
+    if (!q || !k_new || !v_new || !k_cache || !v_cache || !page_table || !out)
+      return RPA_ERR_INVALID_ARG;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RPA_ERR_CUDA;
+    DeviceWs &ws = g_ws[dev];
+    std::lock_guard<std::mutex> lock(ws.mu);
+    rc = ensure_init(ws);
+    if (rc) return rc;
+    Slot &slot = ws.slots[ws.next];
+    ws.next = (ws.next + 1) % kSlots;
+
+    const int G = dims->num_q_heads / dims->num_kv_heads;
+    const int64_t per_partial = (int64_t)dims->num_kv_heads * G * (dims->head_dim + 1);
+    rc = grow_slot(slot, hp.layout.total_words, hp.layout.n_partials * per_partial);
+    if (rc) return rc;
+    serialize(hp, slot.host);
+    if (hp.layout.total_words > 0 &&
+        cudaMemcpyAsync(slot.dev, slot.host, hp.layout.total_words * sizeof(int32_t),
+                        cudaMemcpyHostToDevice, stream) != cudaSuccess)
+      return RPA_ERR_CUDA;
+
+    Problem pb{};
+    pb.q = q;
+    pb.k_new = k_new;
+    pb.v_new = v_new;
+    pb.k_cache = k_cache;
+    pb.v_cache = v_cache;
+    pb.page_table = page_table;
+    pb.out = out;
+    pb.lse = lse;
+    pb.err = ws.err;
+    pb.hq = dims->num_q_heads;
+    pb.hkv = dims->num_kv_heads;
+    pb.d = dims->head_dim;
+    pb.p = dims->page_size;
+    pb.num_pages = dims->num_pages;
+    pb.max_pages = dims->max_pages_per_seq;
+    pb.dtype = dims->dtype;
+    pb.causal = causal ? 1 : 0;
+    pb.scale = scale;
+
+    const PlanLayout &L = hp.layout;
+    float *partial_o = slot.partial;
+    float *partial_lse = slot.partial ? slot.partial + L.n_partials * dims->num_kv_heads * G * dims->head_dim : nullptr;
+    cudaError_t e = cudaSuccess;
+    if (L.n_prefill_tiles > 0 && e == cudaSuccess)
+      e = traced(RPA_KERNEL_PREFILL, stream, [&] {
+        return launch_prefill(pb, (const PrefillTile *)(slot.dev + L.prefill_off),
+                              (int)L.n_prefill_tiles, stream);
+      });
+    if (L.n_decode_items > 0 && e == cudaSuccess)
+      e = traced(RPA_KERNEL_DECODE, stream, [&] {
+        return launch_decode(pb, (const DecodeItem *)(slot.dev + L.decode_off),
+                             (int)L.n_decode_items, partial_o, partial_lse, stream);
+      });
+    if (L.n_combine > 0 && e == cudaSuccess)
+      e = traced(RPA_KERNEL_COMBINE, stream, [&] {
+        return launch_combine(pb, (const CombineItem *)(slot.dev + L.combine_off),
+                              (int)L.n_combine, partial_o, partial_lse, stream);
+      });
+    if (L.n_generic_rows > 0 && e == cudaSuccess)
+      e = traced(RPA_KERNEL_GENERIC, stream, [&] {
+        return launch_generic(pb, (const GenericSeq *)(slot.dev + L.generic_off),
+                              (int)L.n_generic_seqs, (int)L.n_generic_rows, stream);
+      });
+    if (cudaEventRecord(slot.done, stream) == cudaSuccess) slot.pending = true;
+    return e == cudaSuccess ? RPA_OK : RPA_ERR_CUDA;
+  } catch (const std::bad_alloc &) {
+    return RPA_ERR_OOM;
+  }
+}
+
+extern "C" RPA_API int rpa_device_status(void *stream_ptr, uint32_t *flags) {
+  if (flags == nullptr) return RPA_ERR_INVALID_ARG;
+  *flags = 0;
+  if (cudaStreamSynchronize((cudaStream_t)stream_ptr) != cudaSuccess) return RPA_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RPA_ERR_CUDA;
+  DeviceWs &ws = g_ws[dev];
+  std::lock_guard<std::mutex> lock(ws.mu);
+  if (!ws.init) return RPA_OK;
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, ws.err, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return RPA_ERR_CUDA;
+  if (cudaMemset(ws.err, 0, sizeof v) != cudaSuccess) return RPA_ERR_CUDA;
+  *flags = v;
+  return RPA_OK;
+}
+
+extern "C" RPA_API int32_t rpa_profile_enable(int32_t on) { return g_profile_on.exchange(on ? 1 : 0); }
+
+extern "C" RPA_API int rpa_profile_read(double *ms, int64_t *launches) {
+  std::lock_guard<std::mutex> lock(g_profile_mu);
+  double acc[RPA_KERNEL_CLASSES] = {0, 0, 0, 0};
+  int64_t cnt[RPA_KERNEL_CLASSES] = {0, 0, 0, 0};
+  int rc = RPA_OK;
+  for (const Traced &t : g_traced) {
+    float v = 0.f;
+    if (cudaEventSynchronize(t.b) != cudaSuccess || cudaEventElapsedTime(&v, t.a, t.b) != cudaSuccess)
+      rc = RPA_ERR_CUDA;
+    acc[t.kind] += v;
+    cnt[t.kind] += 1;
+    g_event_pool.push_back(t.a);
+    g_event_pool.push_back(t.b);
+  }
+  g_traced.clear();
+  for (int k = 0; k < RPA_KERNEL_CLASSES; ++k) {
+    if (ms) ms[k] = acc[k];
+    if (launches) launches[k] = cnt[k];
+  }
+  return rc;
+}

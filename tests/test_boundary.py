@@ -1,0 +1,171 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads and
+exports every function include/rpa.h declares, validation returns the
+documented codes, and the planner's classification and work lists match the
+lengths it was given."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+from ragged_paged_attention_03_b200 import build as B
+from ragged_paged_attention_03_b200 import inputs as I
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def rb():
+    B.build()
+    from ragged_paged_attention_03_b200 import binding
+    return binding
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "rpa.h")).read()
+    return sorted(set(re.findall(r"RPA_API\s+[\w\s\*]*?\b(rpa_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(rb):
+    names = declared_functions()
+    assert {"rpa_forward", "rpa_device_status", "rpa_status_string", "rpa_plan",
+            "rpa_set_option"} <= set(names)
+    lib = rb.library()
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def dims(**kw):
+    from ragged_paged_attention_03_b200 import binding
+    base = dict(num_q_heads=32, num_kv_heads=8, head_dim=128, page_size=16, num_pages=1000,
+                max_pages_per_seq=64, total_q_tokens=0, dtype=1)
+    base.update(kw)
+    return binding.rpa_dims(**base)
+
+
+def plan(rb, q_lens, kv_lens, dist=None, **kw):
+    cu = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+    return rb.rpa_plan(cu, np.array(kv_lens, np.int32), dist,
+                       dims(total_q_tokens=int(cu[-1]), **kw))
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(head_dim=96), 2), (dict(page_size=12), 2), (dict(page_size=4), 2),
+    (dict(num_kv_heads=5), 2), (dict(num_q_heads=64, num_kv_heads=2), 2),
+    (dict(dtype=7), 1), (dict(num_pages=0), 1),
+])
+def test_bad_dims(rb, kw, code):
+    with pytest.raises(rb.RpaError) as e:
+        plan(rb, [1], [10], **kw)
+    assert e.value.code == code
+
+
+def test_bad_lengths(rb):
+    with pytest.raises(rb.RpaError) as e:
+        plan(rb, [5], [4])                      # kv_len < q_len
+    assert e.value.code == 3
+    with pytest.raises(rb.RpaError) as e:
+        plan(rb, [1], [64 * 16 + 1])            # more pages than a table row holds
+    assert e.value.code == 3
+    with pytest.raises(rb.RpaError) as e:       # T disagrees with cu_q_lens
+        rb.rpa_plan(np.array([0, 3], np.int32), np.array([3], np.int32), None,
+                    dims(total_q_tokens=4))
+    assert e.value.code == 3
+    with pytest.raises(rb.RpaError) as e:       # cu_q_lens must start at 0
+        rb.rpa_plan(np.array([1, 3], np.int32), np.array([3], np.int32), None,
+                    dims(total_q_tokens=3))
+    assert e.value.code == 3
+
+
+def test_bad_distribution(rb):
+    with pytest.raises(rb.RpaError) as e:       # a 5-token sequence in the decode range
+        plan(rb, [1, 5], [9, 5], dist=np.array([2, 2, 2], np.int32))
+    assert e.value.code == 4
+    with pytest.raises(rb.RpaError) as e:       # chunked sequence in the prefill range
+        plan(rb, [1, 5], [9, 9], dist=np.array([1, 2, 2], np.int32))
+    assert e.value.code == 4
+    with pytest.raises(rb.RpaError) as e:       # counts do not cover the batch
+        plan(rb, [1, 5], [9, 9], dist=np.array([1, 1, 3], np.int32))
+    assert e.value.code == 4
+    info = plan(rb, [1, 5, 3], [9, 5, 9], dist=np.array([1, 2, 3], np.int32))
+    assert info.num_decode + info.num_generic + info.num_prefill == 3
+
+
+def test_empty_batches(rb):
+    info = plan(rb, [], [])
+    assert info.plan_bytes == 0
+    info = plan(rb, [0, 0], [5, 9])
+    assert info.num_empty == 2 and info.plan_bytes == 0
+
+
+def test_fp32_routes_to_generic(rb):
+    info = plan(rb, [1, 50, 17], [37, 50, 80], dtype=0)
+    assert info.num_generic == 3 and info.num_decode == 0 and info.num_prefill == 0
+
+
+def test_force_generic_option(rb):
+    old = rb.rpa_set_option(rb.RPA_OPT_FORCE_GENERIC, 1)
+    try:
+        info = plan(rb, [1, 50], [37, 50])
+        assert info.num_generic == 2
+    finally:
+        rb.rpa_set_option(rb.RPA_OPT_FORCE_GENERIC, old)
+
+
+def test_decode_chunking(rb):
+    """Decode work items: ceil(kv_len / 16) blocks per sequence, cut into
+    near-equal chunks of at most the chunk size; sequences cut more than
+    once need the combine."""
+    old = rb.rpa_set_option(rb.RPA_OPT_DECODE_CHUNK_BLOCKS, 8)
+    try:
+        info = plan(rb, [1, 1, 1], [16 * 8, 16 * 8 + 1, 5])
+    finally:
+        rb.rpa_set_option(rb.RPA_OPT_DECODE_CHUNK_BLOCKS, old)
+    if info.num_decode == 0:
+        pytest.skip("decode kernel not routed")
+    assert info.decode_items == 1 + 2 + 1
+    assert info.combine_rows == 1 and info.decode_max_splits == 2
+
+
+def test_workload_plans(rb):
+    """Every named workload plans, and each sequence lands in exactly one class."""
+    for name in I.WORKLOADS:
+        dtype, hq, hkv, d, p, _, _, seed, _ = I.WORKLOADS[name]
+        q_lens, kv_lens = I._lengths(name, torch.Generator().manual_seed(seed))
+        pages = max((k + p - 1) // p for k in kv_lens)
+        cu = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+        info = rb.rpa_plan(cu, np.array(kv_lens, np.int32), I.classify(q_lens, kv_lens),
+                           dims(num_q_heads=hq, num_kv_heads=hkv, head_dim=d, page_size=p,
+                                max_pages_per_seq=pages, total_q_tokens=int(cu[-1]),
+                                num_pages=10 ** 7, dtype=dtype))
+        assert info.num_decode + info.num_prefill + info.num_generic + info.num_empty == len(q_lens)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_forward_without_gpu_fails_loudly(rb):
+    """Without a usable device rpa_forward returns RPA_ERR_CUDA (nothing is
+    computed anywhere else)."""
+    lib = rb.library()
+    cu = np.array([0, 1], np.int32)
+    kv = np.array([4], np.int32)
+    d = dims(total_q_tokens=1)
+    fake = ctypes.c_void_p(0x1000)
+    rc = lib.rpa_forward(fake, fake, fake, fake, fake, fake, cu.ctypes.data_as(ctypes.c_void_p),
+                         kv.ctypes.data_as(ctypes.c_void_p), 1, None, 1.0, 1, fake, None,
+                         ctypes.byref(d), None)
+    assert rc == 6
+
+
+def test_forward_rejects_before_touching_device(rb):
+    lib = rb.library()
+    cu = np.array([0, 2], np.int32)
+    kv = np.array([1], np.int32)     # kv_len < q_len
+    d = dims(total_q_tokens=2)
+    fake = ctypes.c_void_p(0x1000)
+    rc = lib.rpa_forward(fake, fake, fake, fake, fake, fake, cu.ctypes.data_as(ctypes.c_void_p),
+                         kv.ctypes.data_as(ctypes.c_void_p), 1, None, 1.0, 1, fake, None,
+                         ctypes.byref(d), None)
+    assert rc == 3
+    assert rb.rpa_status_string(3) == "invalid sequence lengths"
