@@ -162,8 +162,8 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ GPU arm
-def device_problem(name: str, causal, device) -> I.Problem:
-    return I.make_workload(name, device=device, causal=causal, poison=False)
+def device_problem(name: str, causal, device, max_seqs=None) -> I.Problem:
+    return I.make_workload(name, device=device, causal=causal, poison=False, max_seqs=max_seqs)
 
 
 def time_steps(prob, steps, warmup, flush, stream, profile=False):
@@ -352,6 +352,8 @@ def main():
                                            "mixed_96d_4c,long_d256")
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the cpu_baseline sample")
+    ap.add_argument("--max-seqs", type=int, default=None,
+                    help="keep only the first N sequences of each workload (profiler captures)")
     args = ap.parse_args()
     world, rank, local = dist_setup(args)
     n = world
@@ -401,7 +403,7 @@ def main():
     for i, spec in enumerate(wl):
         name, _, opt = spec.partition(":")
         causal = False if opt == "noncausal" else None
-        prob = device_problem(name, causal, dev)
+        prob = device_problem(name, causal, dev, args.max_seqs)
         work = algorithmic(prob)
         if world > 1:
             torch.distributed.barrier()

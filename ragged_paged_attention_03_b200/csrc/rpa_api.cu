@@ -29,7 +29,10 @@ std::atomic<int64_t> g_opt_force_generic{0};
 std::atomic<int64_t> g_opt_disable_prefill_tc{0};
 
 constexpr int kDefaultDecodeChunkBlocks = 64;
-constexpr bool kHaveDecodeKernel = false;
+// 256 blocks of 16 tokens touch at most 4096 / 8 + 1 pages, within the decode
+// kernel's 1024-entry page list.
+constexpr int kMaxDecodeChunkBlocks = 256;
+constexpr bool kHaveDecodeKernel = true;
 constexpr bool kHavePrefillKernel = false;
 
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
@@ -104,6 +107,7 @@ void build_plan(const int32_t *cu, const int32_t *kv, int32_t n, const int32_t *
                 const rpa_dims *d, HostPlan &hp) {
   int64_t chunk = g_opt_decode_chunk.load();
   if (chunk <= 0) chunk = kDefaultDecodeChunkBlocks;
+  chunk = std::min<int64_t>(chunk, kMaxDecodeChunkBlocks);
   for (int32_t s = 0; s < n; ++s) {
     const int32_t ql = cu[s + 1] - cu[s];
     const int32_t kvl = kv[s];

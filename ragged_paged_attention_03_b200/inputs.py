@@ -139,11 +139,14 @@ WORKLOADS = {
 
 
 def make_workload(name: str, device="cpu", causal: Optional[bool] = None, poison: bool = True,
-                  logical: Optional[bool] = None) -> Problem:
-    """One of the named workloads (see the module docstring)."""
+                  logical: Optional[bool] = None, max_seqs: Optional[int] = None) -> Problem:
+    """One of the named workloads (see the module docstring).  ``max_seqs``
+    keeps only the first sequences (smaller cases for profiler captures)."""
     dtype, hq, hkv, d, p, causal_default, vscale, seed, pool = WORKLOADS[name]
     gen = torch.Generator().manual_seed(seed)
     q_lens, kv_lens = _lengths(name, gen)
+    if max_seqs is not None:
+        q_lens, kv_lens = q_lens[:max_seqs], kv_lens[:max_seqs]
     if logical is None:
         logical = name == "tiny_mixed_f32"
     return make_problem(q_lens, kv_lens, num_q_heads=hq, num_kv_heads=hkv, head_dim=d,
