@@ -52,7 +52,9 @@ enum {
                                 max_pages_per_seq; T != total_q_tokens */
   RPA_ERR_DISTRIBUTION = 4,  /* distribution given and inconsistent */
   RPA_ERR_OOM = 5,           /* library workspace could not be allocated */
-  RPA_ERR_CUDA = 6           /* a CUDA call or kernel launch failed */
+  RPA_ERR_CUDA = 6,          /* a CUDA call or kernel launch failed */
+  RPA_ERR_SCRATCH_LIMIT = 7  /* rpa_decode_noalloc: the batch needs more
+                                scratch than its fixed array holds */
 };
 
 /* Bits of the device error word read by rpa_device_status(). */
@@ -197,6 +199,42 @@ RPA_API int32_t rpa_profile_enable(int32_t on);
  * may be NULL).  Returns RPA_OK or RPA_ERR_CUDA.
  */
 RPA_API int rpa_profile_read(double *ms, int64_t *launches);
+
+/*
+ * rpa_decode_noalloc -- decode-only variant of rpa_forward that allocates
+ * nothing.  The pages have no counterpart to this entry point: it exists for
+ * callers that cannot call cudaMalloc at the point where they run attention
+ * (a memory pool or allocator servicing a request, a serving process whose
+ * device memory is fully reserved up front, a hard memory budget), because
+ * rpa_forward grows a per-device workspace on demand.
+ *
+ * Every sequence has exactly one new token: token s belongs to sequence s,
+ * dims->total_q_tokens == num_seqs, kv_lens[s] >= 1 (host), dtype bf16.
+ * Buffers, layouts and results are those of rpa_forward for such a batch
+ * (causal and non-causal coincide for one new token); the new K/V are
+ * stored into the cache by the same kernels.  dev_flags: device uint32 that
+ * receives RPA_DEV_* bits (OR-ed in, never cleared), or NULL to discard them.
+ *
+ * Scratch: all plan and split-KV buffers live in one file-scope device array
+ * of 16 MiB that every GPU loading this part of the library holds until the
+ * process exits.  A batch whose work items, combine rows or partial results
+ * do not fit is rejected with RPA_ERR_SCRATCH_LIMIT before any device work
+ * (about 8192 work items of 1024 tokens; partial results of
+ * num_kv_heads * G * (head_dim + 1) floats per split item within ~15.6 MiB).
+ * No cudaMalloc, cudaFree, cudaMallocHost or other allocating routine is
+ * called.  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the one array and it keeps the
+ * last call's contents: calls that can overlap on the GPU race on it, so the
+ * caller must order them (for example, one stream per device).
+ */
+RPA_API int rpa_decode_noalloc(const void *q, const void *k_new,
+                               const void *v_new, void *k_cache,
+                               void *v_cache, const int32_t *page_table,
+                               const int32_t *kv_lens, int32_t num_seqs,
+                               float scale, void *out, float *lse,
+                               const rpa_dims *dims, uint32_t *dev_flags,
+                               void *stream);
 
 #ifdef __cplusplus
 }

@@ -68,6 +68,10 @@ _lib.rpa_profile_enable.restype = ctypes.c_int32
 _lib.rpa_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
 _lib.rpa_profile_read.restype = ctypes.c_int
 KERNEL_CLASSES = ("generic", "decode", "combine", "prefill")
+_lib.rpa_decode_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _P, _i32, ctypes.c_float, _P, _P,
+                                    ctypes.POINTER(rpa_dims), _P, _P]
+_lib.rpa_decode_noalloc.restype = ctypes.c_int
+RPA_ERR_SCRATCH_LIMIT = 7
 
 
 def library() -> ctypes.CDLL:
@@ -181,3 +185,23 @@ def rpa_profile_read() -> dict:
     if rc != RPA_OK:
         raise RpaError(rc, "rpa_profile_read")
     return {k: (int(n[i]), float(ms[i])) for i, k in enumerate(KERNEL_CLASSES)}
+
+
+def rpa_decode_noalloc(q, k_new, v_new, k_cache, v_cache, page_table, kv_lens, scale: float, out,
+                       lse=None, dev_flags=None, stream=None) -> None:
+    """Calls rpa_decode_noalloc: a decode-only batch (token s is sequence s's
+    one new token) run entirely in the library's fixed scratch array, for
+    callers that must not allocate device memory.  dev_flags: optional int32
+    CUDA tensor of one element that receives the device error bits."""
+    kv = _host_i32(kv_lens)
+    dims = make_dims(q, k_cache, page_table)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    sptr = ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+    rc = _lib.rpa_decode_noalloc(_dev(q, "q"), _dev(k_new, "k_new"), _dev(v_new, "v_new"),
+                                 _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                                 _dev(page_table, "page_table", torch.int32), _hp(kv), len(kv),
+                                 float(scale), _dev(out, "out"), _dev(lse, "lse", torch.float32),
+                                 ctypes.byref(dims), _dev(dev_flags, "dev_flags", torch.int32), sptr)
+    if rc != RPA_OK:
+        raise RpaError(rc, "rpa_decode_noalloc")

@@ -343,6 +343,7 @@ extern "C" RPA_API const char *rpa_status_string(int status) {
     case RPA_ERR_DISTRIBUTION: return "distribution inconsistent with lengths";
     case RPA_ERR_OOM: return "workspace allocation failed";
     case RPA_ERR_CUDA: return "CUDA error";
+    case RPA_ERR_SCRATCH_LIMIT: return "batch exceeds the no-alloc scratch limit";
     default: return "unknown status";
   }
 }
