@@ -19,6 +19,7 @@ struct Problem {
   float *lse;          // may be null
   uint32_t *err;       // device error word (RPA_DEV_* bits)
   int32_t hq, hkv, d, p, num_pages, max_pages, dtype, causal;
+  int32_t total_q;     // T: rows of q, k_new, v_new, out
   float scale;
 };
 

@@ -1,0 +1,506 @@
+// prefill_kernel.cu -- prefill and chunked-prefill attention on the 5th
+// generation tensor cores (tcgen05 + TMEM), with the fused cache update.
+//
+// The pages measure prefill against the matrix units' peak (talk summary,
+// 00:11:09: up to 73 % MFU, 63 % with a causal mask) and fuse the KV-cache
+// write into the attention kernel (00:06:36).  On B200 one CTA computes one
+// 128-row tile of new tokens for one query head:
+//
+//   warps 0-3  softmax: one query row per thread; S rows come out of TMEM
+//              (tcgen05.ld), P goes back into TMEM as bf16 (tcgen05.st),
+//              online softmax in log2 units with a lazily refreshed running
+//              max (O is rescaled only when the max grows by more than 2^8);
+//              epilogue O / l -> bf16, lse; then the tile's share of the
+//              new K/V rows is copied into its cache pages.
+//   warp 4     producer: TMA of the Q tile, then K and V blocks of BN keys:
+//              cached context from the pages (one box per page segment),
+//              new tokens from k_new / v_new.  Rows of a block that hold no
+//              valid key (past the context, past the sequence, bad pages)
+//              are zeroed before the block is released, so stale or NaN
+//              slots never reach the tensor cores.
+//   warp 5     TMEM owner and MMA issuer (one thread): S = Q K^T into one of
+//              two TMEM buffers, then O += P V with P read from TMEM.
+//
+// Keys are ordered as context blocks [0, c) followed by new-token blocks
+// starting at c, so with BN = 128 the causal diagonal of a 128-row tile is
+// exactly one block.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "kernels.h"
+#include "ptx.cuh"
+#include "tma.h"
+
+namespace rpa {
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
+
+template <int D>
+struct PrefillShape {
+  static constexpr int BM = kPrefillTileRows;          // 128 query rows
+  static constexpr int BN = D == 256 ? 64 : 128;       // keys per block
+  static constexpr int NS = 2;                         // K/V stages
+  static constexpr int kHalves = D / 64;
+  static constexpr int kQBytes = kHalves * BM * 128;
+  static constexpr int kKVBytes = kHalves * BN * 128;  // one K or one V block
+  static constexpr int kData = kQBytes + 2 * NS * kKVBytes;
+  static constexpr int kBarriers = 32;
+  // at least 116 KB so that two CTAs never share an SM (each owns all 512
+  // TMEM columns)
+  static constexpr int kSmemUsed = 1024 + kData + kBarriers * 8 + 64;
+  static constexpr int kSmem = kSmemUsed > 116 * 1024 ? kSmemUsed : 116 * 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColS0 = 0, kColS1 = BN, kColO = 2 * BN;
+  static_assert(kColO + D <= kTmemCols, "TMEM budget");
+};
+
+struct Bars {
+  uint64_t q_full;
+  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t fix, drain;
+};
+
+// Bounded wait that also gives up as soon as another role has aborted.
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                         uint32_t *err) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  while (!ptx::mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (ptx::globaltimer() - t0 > ptx::kWaitLimitNs) {
+      *abort_flag = 1;
+      atomicOr(err, RPA_DEV_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
+                   const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_kn,
+                   const __grid_constant__ CUtensorMap tm_vn, const Problem pb,
+                   const PrefillTile *__restrict__ tiles, float scale_log2) {
+  using S = PrefillShape<D>;
+  constexpr int BM = S::BM, BN = S::BN, NS = S::NS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sQ = base;
+  uint8_t *sK = sQ + S::kQBytes;                 // NS blocks
+  uint8_t *sV = sK + NS * S::kKVBytes;           // NS blocks
+  Bars *bars = reinterpret_cast<Bars *>(base + S::kData);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const PrefillTile tile = tiles[blockIdx.y];
+  const int h = blockIdx.x;
+  const int G = pb.hq / pb.hkv;
+  const int hk = h / G;
+  const int c = tile.kv_len - tile.q_len;             // cached context length
+  const int r0 = tile.tile_row;
+  const int n_ctx = (c + BN - 1) / BN;
+  const int n_new = pb.causal ? (r0 + tile.rows + BN - 1) / BN : (tile.q_len + BN - 1) / BN;
+  const int nb = n_ctx + n_new;
+  const int32_t *pt_row = pb.page_table + (size_t)tile.seq * pb.max_pages;
+
+  if (tid == 0) {
+    ptx::mbar_init(&bars->q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&bars->k_full[i], 1);
+      ptx::mbar_init(&bars->k_empty[i], 1);
+      ptx::mbar_init(&bars->v_full[i], 1);
+      ptx::mbar_init(&bars->v_empty[i], 1);
+      ptx::mbar_init(&bars->s_full[i], 1);
+      ptx::mbar_init(&bars->p_full[i], 128);
+      ptx::mbar_init(&bars->pv_done[i], 1);
+    }
+    ptx::mbar_init(&bars->fix, 1);
+    ptx::mbar_init(&bars->drain, 1);
+    *abort_flag = 0;
+    ptx::fence_barrier_init();
+  }
+  if (warp == 5) {
+    ptx::tmem_alloc(tmem_slot, S::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    ptx::tma_prefetch_desc(&tm_q);
+    ptx::tma_prefetch_desc(&tm_kc);
+    ptx::tma_prefetch_desc(&tm_vc);
+    ptx::tma_prefetch_desc(&tm_kn);
+    ptx::tma_prefetch_desc(&tm_vn);
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    const int br = pb.p < BN ? pb.p : BN;      // rows per page-segment box
+    const int nseg = BN / br;                  // <= 16
+    uint32_t fix_phase = 0;
+    int issued = 0;                            // blocks whose copies were queued
+    if (lane == 0) {
+      ptx::mbar_arrive_expect_tx(&bars->q_full, S::kQBytes);
+      for (int hh = 0; hh < S::kHalves; ++hh)
+        ptx::tma_load_3d(sQ + hh * BM * 128, &tm_q, &bars->q_full, hh * 64, h, tile.q_start + r0);
+    }
+    for (int j = 0; j < nb; ++j) {
+      const int s = j % NS;
+      const uint32_t ph = (uint32_t)((j / NS) & 1);
+      uint8_t *dk = sK + s * S::kKVBytes;
+      uint8_t *dv = sV + s * S::kKVBytes;
+      // Block geometry: valid rows; for context blocks the page of each
+      // segment (lane sg reads segment sg's page-table entry).
+      const bool ctx = j < n_ctx;
+      const int pos0 = ctx ? j * BN : (j - n_ctx) * BN;   // first position / new-token index
+      const int valid = min(BN, (ctx ? c : tile.q_len) - pos0);
+      int page = -1;
+      bool seg_loaded = false, seg_bad = false;
+      if (ctx && lane < nseg) {
+        const int sp = pos0 + lane * br;
+        if (sp < c) {
+          page = pt_row[sp / pb.p];
+          if (page < 0 || page >= pb.num_pages) {
+            seg_bad = true;
+            atomicOr(pb.err, RPA_DEV_BAD_PAGE);
+          } else {
+            seg_loaded = true;
+          }
+        }
+      }
+      const unsigned loaded_mask = __ballot_sync(0xffffffffu, seg_loaded);
+      const bool fix = valid < BN || __any_sync(0xffffffffu, seg_bad);
+      const uint32_t seg_bytes = (uint32_t)(S::kHalves * br * 128);
+      const uint32_t blk_bytes = ctx ? (uint32_t)__popc(loaded_mask) * seg_bytes : (uint32_t)S::kKVBytes;
+
+      if (j >= NS) {
+        if (!wait_bar(&bars->k_empty[s], ph ^ 1u, abort_flag, pb.err)) break;
+        if (!wait_bar(&bars->v_empty[s], ph ^ 1u, abort_flag, pb.err)) break;
+      }
+      if (lane == 0) {
+        uint64_t *kb = fix ? &bars->fix : &bars->k_full[s];
+        uint64_t *vb = fix ? &bars->fix : &bars->v_full[s];
+        if (fix) {
+          ptx::mbar_arrive_expect_tx(&bars->fix, 2 * blk_bytes);
+        } else {
+          ptx::mbar_arrive_expect_tx(&bars->k_full[s], blk_bytes);
+          ptx::mbar_arrive_expect_tx(&bars->v_full[s], blk_bytes);
+        }
+        if (!ctx) {
+          const int row = tile.q_start + pos0;
+          for (int hh = 0; hh < S::kHalves; ++hh) {
+            ptx::tma_load_3d(dk + hh * BN * 128, &tm_kn, kb, hh * 64, hk, row);
+            ptx::tma_load_3d(dv + hh * BN * 128, &tm_vn, vb, hh * 64, hk, row);
+          }
+        }
+      }
+      if (ctx) {
+        // every lane takes part in the broadcast of segment sg's page id;
+        // lane 0 queues the copies
+        for (int sg = 0; sg < nseg; ++sg) {
+          const int pg = __shfl_sync(0xffffffffu, page, sg);
+          if (lane != 0 || !((loaded_mask >> sg) & 1u)) continue;
+          uint64_t *kb = fix ? &bars->fix : &bars->k_full[s];
+          uint64_t *vb = fix ? &bars->fix : &bars->v_full[s];
+          const int sp = pos0 + sg * br;
+          const int row = pg * pb.p + (sp % pb.p);
+          for (int hh = 0; hh < S::kHalves; ++hh) {
+            ptx::tma_load_3d(dk + hh * BN * 128 + sg * br * 128, &tm_kc, kb, hh * 64, hk, row);
+            ptx::tma_load_3d(dv + hh * BN * 128 + sg * br * 128, &tm_vc, vb, hh * 64, hk, row);
+          }
+        }
+      }
+      ++issued;
+      if (fix) {
+        // Wait for this block's copies (the private barrier completes even
+        // with no copies: the arrival carried zero expected bytes), zero
+        // every row that holds no valid key, then publish the block.
+        const bool ok = wait_bar(&bars->fix, fix_phase, abort_flag, pb.err);
+        fix_phase ^= 1u;
+        if (!ok) break;
+        for (int r = lane; r < BN; r += 32) {
+          const bool bad_row = r >= valid || (ctx && !((loaded_mask >> (r / br)) & 1u));
+          if (!bad_row) continue;
+          for (int hh = 0; hh < S::kHalves; ++hh) {
+            uint4 *pk = reinterpret_cast<uint4 *>(dk + hh * BN * 128 + r * 128);
+            uint4 *pv = reinterpret_cast<uint4 *>(dv + hh * BN * 128 + r * 128);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              pk[q] = make_uint4(0, 0, 0, 0);
+              pv[q] = make_uint4(0, 0, 0, 0);
+            }
+          }
+        }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          ptx::mbar_arrive(&bars->k_full[s]);
+          ptx::mbar_arrive(&bars->v_full[s]);
+        }
+      }
+    }
+    // Before the CTA can end, every copy this warp queued must have landed
+    // (bounded waits; they complete without any other warp).
+    if (lane == 0) {
+      ptx::mbar_wait(&bars->q_full, 0);
+      for (int j = issued - NS < 0 ? 0 : issued - NS; j < issued; ++j) {
+        ptx::mbar_wait(&bars->k_full[j % NS], (uint32_t)((j / NS) & 1));
+        ptx::mbar_wait(&bars->v_full[j % NS], (uint32_t)((j / NS) & 1));
+      }
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t tS[2] = {tmem + S::kColS0, tmem + S::kColS1};
+      const uint32_t tO = tmem + S::kColO;
+      constexpr uint32_t idesc_qk = ptx::umma_idesc_bf16(128, BN, false);
+      constexpr uint32_t idesc_pv = ptx::umma_idesc_bf16(128, D, true);
+      const uint32_t q_addr = ptx::smem_u32(sQ);
+      const uint32_t k_addr = ptx::smem_u32(sK);
+      const uint32_t v_addr = ptx::smem_u32(sV);
+      bool ok = wait_bar(&bars->q_full, 0, abort_flag, pb.err);
+      auto pv = [&](int i) -> bool {
+        const int b = i & 1, s = i % NS;
+        if (!wait_bar(&bars->p_full[b], (uint32_t)((i >> 1) & 1), abort_flag, pb.err)) return false;
+        if (!wait_bar(&bars->v_full[s], (uint32_t)((i / NS) & 1), abort_flag, pb.err)) return false;
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t bdesc = ptx::umma_desc_sw128(v_addr + s * S::kKVBytes + kk * 16 * 128, BN * 128, 1024);
+          ptx::umma_ts(tO, tS[b] + kk * 8, bdesc, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        ptx::umma_commit(&bars->pv_done[b]);
+        ptx::umma_commit(&bars->v_empty[s]);
+        return true;
+      };
+      for (int j = 0; ok && j < nb; ++j) {
+        const int b = j & 1, s = j % NS;
+        if (j >= 2 && !wait_bar(&bars->pv_done[b], (uint32_t)(((j - 2) >> 1) & 1), abort_flag, pb.err)) {
+          ok = false;
+          break;
+        }
+        if (!wait_bar(&bars->k_full[s], (uint32_t)((j / NS) & 1), abort_flag, pb.err)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks & 3) * 32;   // 16 bf16 = 32 bytes inside a 128-byte row
+          const uint64_t adesc = ptx::umma_desc_sw128(q_addr + (ks >> 2) * BM * 128 + off, 16, 1024);
+          const uint64_t bdesc = ptx::umma_desc_sw128(k_addr + s * S::kKVBytes + (ks >> 2) * BN * 128 + off, 16, 1024);
+          ptx::umma_ss(tS[b], adesc, bdesc, idesc_qk, ks > 0 ? 1u : 0u);
+        }
+        ptx::umma_commit(&bars->s_full[b]);
+        ptx::umma_commit(&bars->k_empty[s]);
+        if (j >= 1 && !pv(j - 1)) {
+          ok = false;
+          break;
+        }
+      }
+      if (ok) pv(nb - 1);
+      // drain: wait until every MMA this thread issued has completed
+      ptx::umma_commit(&bars->drain);
+      ptx::mbar_wait(&bars->drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------- softmax
+    const int row = tid;                           // 0..127 == TMEM lane
+    const int rn = r0 + row;                       // new-token index of this row
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nb; ++j) {
+      const int b = j & 1;
+      // warp-uniform decisions only: the tcgen05 loads and stores below are
+      // warp-collective
+      if (!__all_sync(0xffffffffu, wait_bar(&bars->s_full[b], (uint32_t)((j >> 1) & 1), abort_flag, pb.err))) {
+        ok = false;
+        break;
+      }
+      ptx::tc_fence_after();
+      const uint32_t tS = lane_base + (b ? S::kColS1 : S::kColS0);
+      float x[BN];
+      {
+        uint32_t r[BN];
+#pragma unroll
+        for (int cc = 0; cc < BN / 32; ++cc)
+          ptx::tmem_ld32(tS + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[cc * 32]));
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < BN; ++i) x[i] = __uint_as_float(r[i]) * scale_log2;
+      }
+      // visible keys of this row in this block: the first `lim` columns
+      const bool ctx = j < n_ctx;
+      int lim;
+      if (ctx) {
+        lim = min(BN, c - j * BN);
+      } else {
+        const int kn0 = (j - n_ctx) * BN;
+        const int end = pb.causal ? min(tile.q_len, rn + 1) : tile.q_len;
+        lim = max(0, min(BN, end - kn0));
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < BN; ++i) {
+        if (i >= lim) x[i] = -INFINITY;
+        mx = fmaxf(mx, x[i]);
+      }
+      const float m_new = fmaxf(m, mx);
+      const bool need = m == -INFINITY ? false : (m_new > m + kRescaleThreshold);
+      float alpha = 1.f;
+      if (__any_sync(0xffffffffu, need)) {
+        // O must hold every earlier block before it is rescaled
+        if (j >= 1 && !__all_sync(0xffffffffu, wait_bar(&bars->pv_done[(j - 1) & 1],
+                                                          (uint32_t)(((j - 1) >> 1) & 1), abort_flag, pb.err))) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        alpha = (m_new == m) ? 1.f : ptx::ex2(m - m_new);
+        if (j >= 1) {
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t r[32];
+            ptx::tmem_ld32(lane_base + S::kColO + cc * 32, r);
+            ptx::tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            ptx::tmem_st32(lane_base + S::kColO + cc * 32, r);
+          }
+          ptx::tmem_st_wait();
+        }
+        m = m_new;
+      } else if (m == -INFINITY) {
+        m = m_new;
+      }
+      const float m_use = m == -INFINITY ? 0.f : m;
+      float sum = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < BN / 64; ++cc) {
+        uint32_t r[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = ptx::ex2(x[cc * 64 + 2 * i] - m_use);
+          const float p1 = ptx::ex2(x[cc * 64 + 2 * i + 1] - m_use);
+          sum += p0 + p1;
+          r[i] = ptx::pack_bf16(p0, p1);
+        }
+        ptx::tmem_st32(tS + cc * 32, r);
+      }
+      ptx::tmem_st_wait();
+      l = l * alpha + sum;
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&bars->p_full[b]);
+    }
+    // epilogue: O / l
+    if (ok && __all_sync(0xffffffffu, wait_bar(&bars->pv_done[(nb - 1) & 1], (uint32_t)(((nb - 1) >> 1) & 1),
+                                                abort_flag, pb.err))) {
+      ptx::tc_fence_after();
+      const float inv = 1.f / l;
+      const bool store = row < tile.rows;
+      __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(pb.out) +
+                           ((size_t)(tile.q_start + rn) * pb.hq + h) * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t r[32];
+        ptx::tmem_ld32(lane_base + S::kColO + cc * 32, r);
+        ptx::tmem_ld_wait();
+        if (store) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = ptx::pack_bf16(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+          uint4 *dst = reinterpret_cast<uint4 *>(out + cc * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+      }
+      if (store && pb.lse != nullptr) pb.lse[(size_t)(tile.q_start + rn) * pb.hq + h] = (m + log2f(l)) * kLn2;
+    }
+    // Fused cache update: the G CTAs of this KV head split the tile's new
+    // rows between them; each row's K and V are copied into its page slot.
+    {
+      const int g = h % G;
+      const int ra = (g * tile.rows) / G, rb = ((g + 1) * tile.rows) / G;
+      const int chunks = D / 8;   // 16-byte chunks per row
+      const __nv_bfloat16 *kn = reinterpret_cast<const __nv_bfloat16 *>(pb.k_new);
+      const __nv_bfloat16 *vn = reinterpret_cast<const __nv_bfloat16 *>(pb.v_new);
+      __nv_bfloat16 *kc = reinterpret_cast<__nv_bfloat16 *>(pb.k_cache);
+      __nv_bfloat16 *vc = reinterpret_cast<__nv_bfloat16 *>(pb.v_cache);
+      for (int idx = tid; idx < (rb - ra) * chunks; idx += 128) {
+        const int r = ra + idx / chunks, ch = idx % chunks;
+        const int i = r0 + r;                  // new-token index
+        const int pos = c + i;
+        const int pg = pt_row[pos / pb.p];
+        if (pg < 0 || pg >= pb.num_pages) {
+          if (ch == 0) atomicOr(pb.err, RPA_DEV_BAD_PAGE);
+          continue;
+        }
+        const size_t src = ((size_t)(tile.q_start + i) * pb.hkv + hk) * D + ch * 8;
+        const size_t dst = (((size_t)pg * pb.p + pos % pb.p) * pb.hkv + hk) * D + ch * 8;
+        *reinterpret_cast<uint4 *>(kc + dst) = *reinterpret_cast<const uint4 *>(kn + src);
+        *reinterpret_cast<uint4 *>(vc + dst) = *reinterpret_cast<const uint4 *>(vn + src);
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == 5) ptx::tmem_dealloc(tmem, S::kTmemCols);
+}
+
+template <int D>
+cudaError_t launch_prefill_t(const Problem &pb, const PrefillTile *tiles, int n_tiles, cudaStream_t stream) {
+  using S = PrefillShape<D>;
+  CUtensorMap tq, tkc, tvc, tkn, tvn;
+  const uint64_t qdims[3] = {(uint64_t)D, (uint64_t)pb.hq, (uint64_t)pb.total_q};
+  const uint64_t qstr[2] = {(uint64_t)D * 2, (uint64_t)pb.hq * D * 2};
+  const uint32_t qbox[3] = {64, 1, (uint32_t)S::BM};
+  const uint64_t cdims[3] = {(uint64_t)D, (uint64_t)pb.hkv, (uint64_t)pb.num_pages * pb.p};
+  const uint64_t cstr[2] = {(uint64_t)D * 2, (uint64_t)pb.hkv * D * 2};
+  const uint32_t cbox[3] = {64, 1, (uint32_t)(pb.p < S::BN ? pb.p : S::BN)};
+  const uint64_t ndims[3] = {(uint64_t)D, (uint64_t)pb.hkv, (uint64_t)pb.total_q};
+  const uint64_t nstr[2] = {(uint64_t)D * 2, (uint64_t)pb.hkv * D * 2};
+  const uint32_t nbox[3] = {64, 1, (uint32_t)S::BN};
+  if (!make_tmap_bf16_3d(&tq, pb.q, qdims, qstr, qbox, true) ||
+      !make_tmap_bf16_3d(&tkc, pb.k_cache, cdims, cstr, cbox, true) ||
+      !make_tmap_bf16_3d(&tvc, pb.v_cache, cdims, cstr, cbox, true) ||
+      !make_tmap_bf16_3d(&tkn, pb.k_new, ndims, nstr, nbox, true) ||
+      !make_tmap_bf16_3d(&tvn, pb.v_new, ndims, nstr, nbox, true))
+    return cudaErrorInvalidValue;
+  auto kern = prefill_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)pb.hq, (unsigned)n_tiles);
+  kern<<<grid, 192, S::kSmem, stream>>>(tq, tkc, tvc, tkn, tvn, pb, tiles, pb.scale * kLog2e);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const Problem &pb, const PrefillTile *tiles, int n_tiles, cudaStream_t stream) {
+  if (n_tiles <= 0) return cudaSuccess;
+  switch (pb.d) {
+    case 64: return launch_prefill_t<64>(pb, tiles, n_tiles, stream);
+    case 128: return launch_prefill_t<128>(pb, tiles, n_tiles, stream);
+    case 256: return launch_prefill_t<256>(pb, tiles, n_tiles, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace rpa

@@ -33,7 +33,7 @@ constexpr int kDefaultDecodeChunkBlocks = 64;
 // kernel's 1024-entry page list.
 constexpr int kMaxDecodeChunkBlocks = 256;
 constexpr bool kHaveDecodeKernel = true;
-constexpr bool kHavePrefillKernel = false;
+constexpr bool kHavePrefillKernel = true;
 
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
@@ -432,6 +432,7 @@ extern "C" RPA_API int rpa_forward(const void *q, const void *k_new, const void 
     pb.dtype = dims->dtype;
     pb.causal = causal ? 1 : 0;
     pb.scale = scale;
+    pb.total_q = T;
 
     const PlanLayout &L = hp.layout;
     float *partial_o = slot.partial;
