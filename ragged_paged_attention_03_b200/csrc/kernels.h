@@ -38,11 +38,19 @@ cudaError_t launch_combine(const Problem &pb, const CombineItem *items,
                            int n_items, const float *partial_o,
                            const float *partial_lse, cudaStream_t stream);
 
-// Prefill / chunked-prefill kernel (bf16, tcgen05): one CTA per (tile, query head).
+// Prefill / chunked-prefill kernel (bf16, tcgen05): one CTA per (tile, query
+// head).  head_dim 256: one 128-row tile per CTA.
 cudaError_t launch_prefill(const Problem &pb, const PrefillTile *tiles,
                            int n_tiles, cudaStream_t stream);
 
-// Rows per prefill tile (query tokens per CTA tile).
+// head_dim 64 / 128: two 128-row tiles per CTA (a 256-row work item).
+cudaError_t launch_prefill2(const Problem &pb, const PrefillTile *tiles,
+                            int n_tiles, cudaStream_t stream);
+
+// Rows of a single prefill tile (query tokens per TMEM accumulator).
 constexpr int kPrefillTileRows = 128;
+
+// Rows of one prefill work item for a head dim.
+inline int prefill_item_rows(int head_dim) { return head_dim <= 128 ? 256 : 128; }
 
 }  // namespace rpa

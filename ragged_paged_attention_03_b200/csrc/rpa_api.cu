@@ -160,14 +160,15 @@ void build_plan(const int32_t *cu, const int32_t *kv, int32_t n, const int32_t *
       }
       case kPrefill: {
         ++hp.num_prefill;
-        for (int32_t r = 0; r < ql; r += kPrefillTileRows) {
+        const int32_t item_rows = prefill_item_rows(d->head_dim);
+        for (int32_t r = 0; r < ql; r += item_rows) {
           PrefillTile t{};
           t.seq = s;
           t.q_start = cu[s];
           t.q_len = ql;
           t.kv_len = kvl;
           t.tile_row = r;
-          t.rows = std::min(kPrefillTileRows, ql - r);
+          t.rows = std::min(item_rows, ql - r);
           hp.prefill.push_back(t);
         }
         break;
@@ -440,8 +441,9 @@ extern "C" RPA_API int rpa_forward(const void *q, const void *k_new, const void 
     cudaError_t e = cudaSuccess;
     if (L.n_prefill_tiles > 0 && e == cudaSuccess)
       e = traced(RPA_KERNEL_PREFILL, stream, [&] {
-        return launch_prefill(pb, (const PrefillTile *)(slot.dev + L.prefill_off),
-                              (int)L.n_prefill_tiles, stream);
+        const PrefillTile *tiles = (const PrefillTile *)(slot.dev + L.prefill_off);
+        return pb.d <= 128 ? launch_prefill2(pb, tiles, (int)L.n_prefill_tiles, stream)
+                           : launch_prefill(pb, tiles, (int)L.n_prefill_tiles, stream);
       });
     if (L.n_decode_items > 0 && e == cudaSuccess)
       e = traced(RPA_KERNEL_DECODE, stream, [&] {
