@@ -11,19 +11,19 @@
 //   warp 8                   TMA producer: Q tiles, then K/V blocks of 128
 //                            keys (context from pages, new tokens from
 //                            k_new / v_new; rows without a valid key zeroed)
-//   warp 9                   TMEM owner, single-thread tcgen05.mma issue
+//   warp 9                   TMEM owner and MMA issue
 //   warps 10-11              fused cache update: this CTA's share of the new
 //                            K/V rows copied into their page slots
+// The producer and MMA warps run their loops with all 32 lanes and let one
+// elected lane issue each TMA copy, MMA, commit and arrive: a single-lane
+// branch would keep the operands in per-thread registers and cost many issue
+// slots per MMA while the softmax warps keep the sub-partitions busy.
 //
 // TMEM (512 columns): S/P of tile 0 | S/P of tile 1 | O of tile 0 | O of tile 1.
-// P overwrites its tile's S as bf16 and is the A operand of O += P V.  MMA
-// issue order per key block j: PV(0,j), QK(0,j+1), PV(1,j), QK(1,j+1).
+// P overwrites its tile's S as bf16 and is the A operand of O += P V.  The
+// tensor pipe sees QK(0,j+1), PV(1,j), QK(1,j+1), PV(0,j+1), ...: while one
+// tile's softmax runs, the other tile's PV and QK execute.
 //
-// exp2 on the multi-function unit is the softmax bottleneck on this part, so
-// a quarter of the exponentials are computed on the FMA pipe instead: round
-// x to the nearest integer n, f = x - n in [-1/2, 1/2], 2^f by a degree-3
-// polynomial fitted for minimax relative error (max 7.5e-5, far below the
-// bf16 rounding of P), and 2^n added into the exponent field.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <math.h>
@@ -75,37 +75,9 @@ __device__ __forceinline__ bool wait_bar2(uint64_t *bar, uint32_t parity, volati
   return true;
 }
 
-// 2^x for x <= ~8 on the FMA pipe (see the file comment).
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -125.0f);                   // keeps n >= -125: 2^n stays a normal number
-  const float r = x + 12582912.0f;          // 1.5 * 2^23: x rounded to nearest in the low bits
-  const float n = r - 12582912.0f;
-  const float f = x - n;
-  float p = fmaf(0.0551709607f, f, 0.242609662f);
-  p = fmaf(p, f, 0.693260965f);
-  p = fmaf(p, f, 0.999928165f);
-  const int ni = __float_as_int(r) - 0x4B400000;
-  return __int_as_float(__float_as_int(p) + (ni << 23));
-}
-
-// The same on a packed pair: (x0, x1) -> (2^x0, 2^x1), with x already
-// clamped to >= -125.
-__device__ __forceinline__ uint64_t exp2_fma2(float x0, float x1) {
-  const uint64_t x = ptx::f2_pack(x0, x1);
-  const uint64_t magic = ptx::f2_pack(12582912.0f, 12582912.0f);
-  const uint64_t neg_magic = ptx::f2_pack(-12582912.0f, -12582912.0f);
-  const uint64_t r = ptx::f2_add(x, magic);
-  const uint64_t n = ptx::f2_add(r, neg_magic);
-  const uint64_t f = ptx::f2_fma(n, ptx::f2_pack(-1.0f, -1.0f), x);
-  uint64_t p = ptx::f2_fma(ptx::f2_pack(0.0551709607f, 0.0551709607f), f, ptx::f2_pack(0.242609662f, 0.242609662f));
-  p = ptx::f2_fma(p, f, ptx::f2_pack(0.693260965f, 0.693260965f));
-  p = ptx::f2_fma(p, f, ptx::f2_pack(0.999928165f, 0.999928165f));
-  float r0, r1, p0, p1;
-  ptx::f2_unpack(r, r0, r1);
-  ptx::f2_unpack(p, p0, p1);
-  const int n0 = __float_as_int(r0) - 0x4B400000, n1 = __float_as_int(r1) - 0x4B400000;
-  return ptx::f2_pack(__int_as_float(__float_as_int(p0) + (n0 << 23)),
-                      __int_as_float(__float_as_int(p1) + (n1 << 23)));
+// wait_bar2 by every lane of a warp, with a warp-uniform result.
+__device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity, volatile int *abort_flag, uint32_t *err) {
+  return __all_sync(0xffffffffu, wait_bar2(bar, parity, abort_flag, err));
 }
 
 __device__ __forceinline__ void setmaxnreg_inc200() {
@@ -140,6 +112,125 @@ __device__ __forceinline__ Unit make_unit(const PrefillTile *tiles, int u, const
   }
   w.nb = max(w.n_t[0], w.n_t[1]);
   return w;
+}
+
+// QK(t, gblk): S of tile t = Q_t K^T for K/V block gblk (stage gblk % NS).
+template <int D>
+__device__ __forceinline__ bool issue_qk(Bars2 *bars, volatile int *abort_flag, uint32_t *err, uint32_t tS,
+                                         uint64_t dq, uint64_t dk0, int gblk, bool wait_k) {
+  using S = P2Shape<D>;
+  constexpr uint32_t idesc = ptx::umma_idesc_bf16(128, S::BN, false);
+  const int s = gblk % S::NS;
+  if (wait_k && !wait_all(&bars->k_full[s], (uint32_t)((gblk / S::NS) & 1), abort_flag, err)) return false;
+  ptx::tc_fence_after();
+  const uint64_t dk = dk0 + (uint64_t)((s * S::kKVBytes) >> 4);
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks) {
+    const uint32_t offq = ((ks >> 2) * S::BM * 128 + (ks & 3) * 32) >> 4;
+    const uint32_t offk = ((ks >> 2) * S::BN * 128 + (ks & 3) * 32) >> 4;
+    ptx::umma_ss_elect(tS, dq + offq, dk + offk, idesc, ks > 0 ? 1u : 0u);
+  }
+  return true;
+}
+
+// PV(t, gblk): O_t (+)= P_t V for K/V block gblk; P_t is read from TMEM.
+template <int D>
+__device__ __forceinline__ bool issue_pv(Bars2 *bars, volatile int *abort_flag, uint32_t *err, int t,
+                                         uint32_t tS, uint32_t tO, uint64_t dv0, int gblk, int tblk,
+                                         bool first, bool wait_v) {
+  using S = P2Shape<D>;
+  constexpr uint32_t idesc = ptx::umma_idesc_bf16(128, D, true);
+  const int s = gblk % S::NS;
+  if (!wait_all(&bars->p_full[t], (uint32_t)(tblk & 1), abort_flag, err)) return false;
+  if (wait_v && !wait_all(&bars->v_full[s], (uint32_t)((gblk / S::NS) & 1), abort_flag, err)) return false;
+  ptx::tc_fence_after();
+  const uint64_t dv = dv0 + (uint64_t)((s * S::kKVBytes) >> 4);
+#pragma unroll
+  for (int kk = 0; kk < S::BN / 16; ++kk)
+    ptx::umma_ts_elect(tO, tS + kk * 8, dv + (uint64_t)((kk * 16 * 128) >> 4), idesc, (!first || kk > 0) ? 1u : 0u);
+  return true;
+}
+
+// The MMA warp (all 32 lanes; one elected lane issues).  Per unit, with the
+// two tiles' chains interleaved (the tensor pipe sees QK0, PV1, QK1, PV0,
+// ...):
+//   prologue  QK(0,0) QK(1,0) PV(0,0)
+//   block j   QK(0,j+1) PV(1,j) QK(1,j+1) PV(0,j+1)
+// A QK into tile t's S/P columns is issued right after the PV that reads P
+// from them, without waiting for that PV to finish: tcgen05.mma operations
+// issued by one thread execute in issue order.  The same order makes
+// s_full(t, j+1) (committed after QK(t, j+1)) imply that PV(t, j) is
+// complete, which the softmax warps rely on before rescaling O.
+template <int D>
+__device__ __forceinline__ void mma_loop(Bars2 *bars, volatile int *abort_flag, const Problem pb,
+                                         const PrefillTile *tiles, int n_units, uint32_t tmem, uint32_t q_addr,
+                                         uint32_t k_addr, uint32_t v_addr) {
+  using S = P2Shape<D>;
+  constexpr int BM = S::BM, BN = S::BN, NS = S::NS;
+  const uint32_t tS0 = tmem, tS1 = tmem + 128;
+  const uint32_t tO0 = tmem + S::kColO, tO1 = tmem + S::kColO + D;
+  // Descriptors of the stage-0 / tile-0 operands; the start-address field
+  // is the low 14 bits (address / 16), so stages, tiles, k-steps and column
+  // tiles are reached by adding (byte offset / 16).
+  const uint64_t dq0 = ptx::umma_desc_sw128(q_addr, 16, 1024);
+  const uint64_t dq1 = dq0 + (uint64_t)(S::kQBytes >> 4);
+  const uint64_t dk0 = ptx::umma_desc_sw128(k_addr, 16, 1024);
+  const uint64_t dv0 = ptx::umma_desc_sw128(v_addr, BN * 128, 1024);
+  uint32_t *err = pb.err;
+  int g0 = 0, gt0 = 0, gt1 = 0, ep0 = 0, ep1 = 0, uq = 0;
+  bool ok = true;
+  for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x, ++uq) {
+    const Unit w = make_unit<BM, BN>(tiles, u, pb);
+    const int n0 = w.n_t[0], n1 = w.n_t[1], nb = w.nb;
+    ok = wait_all(&bars->q_full, (uint32_t)(uq & 1), abort_flag, err);
+    // prologue
+    if (ok && n0 > 0) ok = issue_qk<D>(bars, abort_flag, err, tS0, dq0, dk0, g0, true);
+    if (ok && n0 > 0) ptx::umma_commit_elect(&bars->s_full[0]);
+    if (ok && n1 > 0) ok = issue_qk<D>(bars, abort_flag, err, tS1, dq1, dk0, g0, n0 == 0);
+    if (ok && n1 > 0) ptx::umma_commit_elect(&bars->s_full[1]);
+    if (ok) ptx::umma_commit_elect(&bars->k_empty[g0 % NS]);
+    if (ok && nb == 1) ptx::umma_commit_elect(&bars->q_empty);
+    if (ok && n0 > 0) {
+      // O_0 is overwritten by the unit's first PV: the softmax warps must
+      // have read the previous unit's O_0
+      if (ep0 > 0) ok = wait_all(&bars->o_free[0], (uint32_t)((ep0 - 1) & 1), abort_flag, err);
+      if (ok) ok = issue_pv<D>(bars, abort_flag, err, 0, tS0, tO0, dv0, g0, gt0, true, true);
+      // pv_done is waited for only after a tile's last block (epilogue)
+      if (ok && n0 == 1) ptx::umma_commit_elect(&bars->pv_done[0]);
+    }
+    for (int j = 0; ok && j < nb; ++j) {
+      const bool k_next_waited = j + 1 < n0;
+      if (j + 1 < n0) {
+        ok = issue_qk<D>(bars, abort_flag, err, tS0, dq0, dk0, g0 + j + 1, true);
+        if (ok) ptx::umma_commit_elect(&bars->s_full[0]);
+      }
+      if (ok && j < n1) {
+        if (j == 0 && ep1 > 0) ok = wait_all(&bars->o_free[1], (uint32_t)((ep1 - 1) & 1), abort_flag, err);
+        // V(j) was already waited for by PV(0, j) when tile 0 used block j
+        if (ok) ok = issue_pv<D>(bars, abort_flag, err, 1, tS1, tO1, dv0, g0 + j, gt1 + j, j == 0, j >= n0);
+        if (ok && j + 1 == n1) ptx::umma_commit_elect(&bars->pv_done[1]);
+      }
+      if (ok) ptx::umma_commit_elect(&bars->v_empty[(g0 + j) % NS]);   // both PVs of block j issued
+      if (ok && j + 1 < n1) {
+        ok = issue_qk<D>(bars, abort_flag, err, tS1, dq1, dk0, g0 + j + 1, !k_next_waited);
+        if (ok) ptx::umma_commit_elect(&bars->s_full[1]);
+      }
+      if (ok && j + 1 < nb) ptx::umma_commit_elect(&bars->k_empty[(g0 + j + 1) % NS]);
+      if (ok && j + 2 == nb) ptx::umma_commit_elect(&bars->q_empty);   // last QK of the unit issued
+      if (ok && j + 1 < n0) {
+        ok = issue_pv<D>(bars, abort_flag, err, 0, tS0, tO0, dv0, g0 + j + 1, gt0 + j + 1, false, true);
+        if (ok && j + 2 == n0) ptx::umma_commit_elect(&bars->pv_done[0]);
+      }
+    }
+    g0 += nb;
+    gt0 += n0;
+    gt1 += n1;
+    ep0 += n0 > 0 ? 1 : 0;
+    ep1 += n1 > 0 ? 1 : 0;
+  }
+  ptx::umma_commit_elect(&bars->drain);
+  ptx::mbar_wait(&bars->drain, 0);
+  __syncwarp();
 }
 
 // Persistent: CTA b handles units b, b + gridDim.x, ... of the list of
@@ -220,15 +311,13 @@ __global__ void __launch_bounds__(384, 1)
         const Unit w = make_unit<BM, BN>(tiles, u, pb);
         const int32_t *pt_row = pb.page_table + (size_t)w.tile.seq * pb.max_pages;
         // Q of both tiles, once the previous unit's QK MMAs are done with sQ
-        if (uq > 0 && !wait_bar2(&bars->q_empty, (uint32_t)((uq - 1) & 1), abort_flag, pb.err)) break;
-        if (lane == 0) {
-          ptx::mbar_arrive_expect_tx(&bars->q_full, (w.rows_t[1] > 0 ? 2 : 1) * S::kQBytes);
-          for (int t = 0; t < 2; ++t) {
-            if (w.rows_t[t] == 0) continue;
-            for (int hh = 0; hh < S::kHalves; ++hh)
-              ptx::tma_load_3d(sQ + t * S::kQBytes + hh * BM * 128, &tm_q, &bars->q_full, hh * 64, w.h,
-                               w.tile.q_start + w.r0 + t * BM);
-          }
+        if (uq > 0 && !wait_all(&bars->q_empty, (uint32_t)((uq - 1) & 1), abort_flag, pb.err)) break;
+        ptx::mbar_arrive_expect_tx_elect(&bars->q_full, (w.rows_t[1] > 0 ? 2 : 1) * S::kQBytes);
+        for (int t = 0; t < 2; ++t) {
+          if (w.rows_t[t] == 0) continue;
+          for (int hh = 0; hh < S::kHalves; ++hh)
+            ptx::tma_load_3d_elect(sQ + t * S::kQBytes + hh * BM * 128, &tm_q, &bars->q_full, hh * 64, w.h,
+                                   w.tile.q_start + w.r0 + t * BM);
         }
         for (int j = 0; j < w.nb; ++j, ++g) {
           const int s = g % NS;
@@ -257,45 +346,42 @@ __global__ void __launch_bounds__(384, 1)
           const uint32_t seg_bytes = (uint32_t)(S::kHalves * br * 128);
           const uint32_t blk_bytes = ctx ? (uint32_t)__popc(loaded_mask) * seg_bytes : (uint32_t)S::kKVBytes;
           if (g >= NS) {
-            if (!wait_bar2(&bars->k_empty[s], ph ^ 1u, abort_flag, pb.err) ||
-                !wait_bar2(&bars->v_empty[s], ph ^ 1u, abort_flag, pb.err)) {
+            if (!wait_all(&bars->k_empty[s], ph ^ 1u, abort_flag, pb.err) ||
+                !wait_all(&bars->v_empty[s], ph ^ 1u, abort_flag, pb.err)) {
               ok = false;
               break;
             }
           }
           uint64_t *kb = fix ? &bars->fix : &bars->k_full[s];
           uint64_t *vb = fix ? &bars->fix : &bars->v_full[s];
-          if (lane == 0) {
-            if (fix) {
-              ptx::mbar_arrive_expect_tx(&bars->fix, 2 * blk_bytes);
-            } else {
-              ptx::mbar_arrive_expect_tx(&bars->k_full[s], blk_bytes);
-              ptx::mbar_arrive_expect_tx(&bars->v_full[s], blk_bytes);
-            }
-            if (!ctx) {
-              const int row = w.tile.q_start + pos0;
-              for (int hh = 0; hh < S::kHalves; ++hh) {
-                ptx::tma_load_3d(dk + hh * BN * 128, &tm_kn, kb, hh * 64, w.hk, row);
-                ptx::tma_load_3d(dv + hh * BN * 128, &tm_vn, vb, hh * 64, w.hk, row);
-              }
-            }
+          if (fix) {
+            ptx::mbar_arrive_expect_tx_elect(&bars->fix, 2 * blk_bytes);
+          } else {
+            ptx::mbar_arrive_expect_tx_elect(&bars->k_full[s], blk_bytes);
+            ptx::mbar_arrive_expect_tx_elect(&bars->v_full[s], blk_bytes);
           }
-          if (ctx) {
+          if (!ctx) {
+            const int row = w.tile.q_start + pos0;
+            for (int hh = 0; hh < S::kHalves; ++hh) {
+              ptx::tma_load_3d_elect(dk + hh * BN * 128, &tm_kn, kb, hh * 64, w.hk, row);
+              ptx::tma_load_3d_elect(dv + hh * BN * 128, &tm_vn, vb, hh * 64, w.hk, row);
+            }
+          } else {
             for (int sg = 0; sg < nseg; ++sg) {
               const int pg = __shfl_sync(0xffffffffu, page, sg);
-              if (lane != 0 || !((loaded_mask >> sg) & 1u)) continue;
+              if (!((loaded_mask >> sg) & 1u)) continue;
               const int sp = pos0 + sg * br;
               const int row = pg * pb.p + (sp % pb.p);
               for (int hh = 0; hh < S::kHalves; ++hh) {
-                ptx::tma_load_3d(dk + hh * BN * 128 + sg * br * 128, &tm_kc, kb, hh * 64, w.hk, row);
-                ptx::tma_load_3d(dv + hh * BN * 128 + sg * br * 128, &tm_vc, vb, hh * 64, w.hk, row);
+                ptx::tma_load_3d_elect(dk + hh * BN * 128 + sg * br * 128, &tm_kc, kb, hh * 64, w.hk, row);
+                ptx::tma_load_3d_elect(dv + hh * BN * 128 + sg * br * 128, &tm_vc, vb, hh * 64, w.hk, row);
               }
             }
           }
           if (fix) {
             // wait for this block's copies (the private barrier completes
             // even with none), zero the rows without a valid key, publish
-            const bool fok = wait_bar2(&bars->fix, fix_phase, abort_flag, pb.err);
+            const bool fok = wait_all(&bars->fix, fix_phase, abort_flag, pb.err);
             fix_phase ^= 1u;
             if (!fok) {
               ok = false;
@@ -317,10 +403,8 @@ __global__ void __launch_bounds__(384, 1)
             }
             ptx::fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) {
-              ptx::mbar_arrive(&bars->k_full[s]);
-              ptx::mbar_arrive(&bars->v_full[s]);
-            }
+            ptx::mbar_arrive_elect(&bars->k_full[s]);
+            ptx::mbar_arrive_elect(&bars->v_full[s]);
           }
         }
       }
@@ -335,96 +419,8 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
     } else if (warp == 9) {
       // --------------------------------------------------------------- MMA
-      if (lane == 0) {
-        const uint32_t tS[2] = {tmem, tmem + 128};
-        const uint32_t tO[2] = {tmem + S::kColO, tmem + S::kColO + D};
-        constexpr uint32_t idesc_qk = ptx::umma_idesc_bf16(128, BN, false);
-        constexpr uint32_t idesc_pv = ptx::umma_idesc_bf16(128, D, true);
-        const uint32_t q_addr = ptx::smem_u32(sQ);
-        const uint32_t k_addr = ptx::smem_u32(sK);
-        const uint32_t v_addr = ptx::smem_u32(sV);
-        int g0 = 0;              // first global block index of the unit
-        int gt[2] = {0, 0};      // blocks of each tile consumed so far
-        int ep[2] = {0, 0};      // units in which each tile was active
-        bool ok = true;
-        // Descriptors of the stage-0 / tile-0 operands; the start-address
-        // field is the low 14 bits (address / 16), so other stages, tiles,
-        // k-steps and column tiles are reached by adding (offset / 16).
-        const uint64_t dq0 = ptx::umma_desc_sw128(q_addr, 16, 1024);
-        const uint64_t dk0 = ptx::umma_desc_sw128(k_addr, 16, 1024);
-        const uint64_t dv0 = ptx::umma_desc_sw128(v_addr, BN * 128, 1024);
-        auto qk = [&](int t, int gblk) -> bool {
-          const int s = gblk % NS;
-          if (!wait_bar2(&bars->k_full[s], (uint32_t)((gblk / NS) & 1), abort_flag, pb.err)) return false;
-          ptx::tc_fence_after();
-          const uint64_t dq = dq0 + (uint64_t)((t * S::kQBytes) >> 4);
-          const uint64_t dk = dk0 + (uint64_t)((s * S::kKVBytes) >> 4);
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = ((ks >> 2) * BM * 128 + (ks & 3) * 32) >> 4;
-            const uint32_t offk = ((ks >> 2) * BN * 128 + (ks & 3) * 32) >> 4;
-            ptx::umma_ss(tS[t], dq + off, dk + offk, idesc_qk, ks > 0 ? 1u : 0u);
-          }
-          ptx::umma_commit(&bars->s_full[t]);
-          return true;
-        };
-        auto pv = [&](int t, int gblk, int tblk, bool first) -> bool {
-          const int s = gblk % NS;
-          if (!wait_bar2(&bars->p_full[t], (uint32_t)(tblk & 1), abort_flag, pb.err)) return false;
-          if (!wait_bar2(&bars->v_full[s], (uint32_t)((gblk / NS) & 1), abort_flag, pb.err)) return false;
-          ptx::tc_fence_after();
-          const uint64_t dv = dv0 + (uint64_t)((s * S::kKVBytes) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)
-            ptx::umma_ts(tO[t], tS[t] + kk * 8, dv + (uint64_t)((kk * 16 * 128) >> 4), idesc_pv,
-                         (!first || kk > 0) ? 1u : 0u);
-          ptx::umma_commit(&bars->pv_done[t]);
-          return true;
-        };
-        int uq = 0;
-        for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x, ++uq) {
-          const Unit w = make_unit<BM, BN>(tiles, u, pb);
-          ok = wait_bar2(&bars->q_full, (uint32_t)(uq & 1), abort_flag, pb.err);
-          // first QK of each tile: its S/P buffer must have been read by the
-          // previous unit's last PV
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            if (!ok || w.n_t[t] == 0) continue;
-            if (gt[t] > 0) ok = wait_bar2(&bars->pv_done[t], (uint32_t)((gt[t] - 1) & 1), abort_flag, pb.err);
-            if (ok) ok = qk(t, g0);
-          }
-          if (ok) ptx::umma_commit(&bars->k_empty[g0 % NS]);
-          if (ok && w.nb == 1) ptx::umma_commit(&bars->q_empty);
-          for (int j = 0; ok && j < w.nb; ++j) {
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-              if (ok && j < w.n_t[t]) {
-                // O of tile t is overwritten by the unit's first PV: the
-                // softmax warps must have read the previous unit's O
-                if (j == 0 && ep[t] > 0)
-                  ok = wait_bar2(&bars->o_free[t], (uint32_t)((ep[t] - 1) & 1), abort_flag, pb.err);
-                if (ok) ok = pv(t, g0 + j, gt[t] + j, j == 0);
-              }
-              if (ok && j + 1 < w.n_t[t]) {
-                ok = wait_bar2(&bars->pv_done[t], (uint32_t)((gt[t] + j) & 1), abort_flag, pb.err);
-                if (ok) ok = qk(t, g0 + j + 1);
-              }
-            }
-            if (ok) ptx::umma_commit(&bars->v_empty[(g0 + j) % NS]);
-            if (ok && j + 1 < w.nb) ptx::umma_commit(&bars->k_empty[(g0 + j + 1) % NS]);
-            if (ok && j + 2 == w.nb) ptx::umma_commit(&bars->q_empty);   // last QK of the unit issued
-          }
-          g0 += w.nb;
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            gt[t] += w.n_t[t];
-            ep[t] += w.n_t[t] > 0 ? 1 : 0;
-          }
-        }
-        ptx::umma_commit(&bars->drain);
-        ptx::mbar_wait(&bars->drain, 0);
-      }
-      __syncwarp();
+      mma_loop<D>(bars, abort_flag, pb, tiles, n_units, tmem, ptx::smem_u32(sQ), ptx::smem_u32(sK),
+                  ptx::smem_u32(sV));
     } else {
       // ------------------------------------------ fused cache update (64 thr)
       const int chunks = D / 8;
@@ -463,6 +459,7 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tS = lane_base + (uint32_t)(t * 128);
     const uint32_t tO = lane_base + S::kColO + (uint32_t)(t * D);
     int gt = 0;                                  // blocks of this tile consumed so far
+    int ep = 0;                                  // units in which this tile had rows
     bool ok = true;
     for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
       const Unit w = make_unit<BM, BN>(tiles, u, pb);
@@ -510,7 +507,8 @@ __global__ void __launch_bounds__(384, 1)
         const bool need = m != -INFINITY && m_new > m + kRescaleThreshold;
         float alpha = 1.f;
         if (__any_sync(0xffffffffu, need)) {
-          // PV(t, j-1) has completed: QK(t, j) was issued only after it.
+          // PV(t, j-1) has completed: s_full(t, j) was committed after QK(t, j),
+          // which was issued after PV(t, j-1).
           alpha = (m_new == m) ? 1.f : ptx::ex2(m - m_new);
           if (j > 0) {
 #pragma unroll 1
@@ -536,17 +534,7 @@ __global__ void __launch_bounds__(384, 1)
         for (int i = 0; i < BN; i += 2) {
           float a0, a1;
           ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(x[i], x[i + 1]), scale2, negm2), a0, a1);
-          uint64_t pp;
-          if ((i & 7) == 6) {          // a quarter of the exponentials on the FMA pipe
-            pp = exp2_fma2(fmaxf(a0, -125.0f), fmaxf(a1, -125.0f));
-            if (masked) {
-              float p0, p1;
-              ptx::f2_unpack(pp, p0, p1);
-              pp = ptx::f2_pack(i < lim ? p0 : 0.f, i + 1 < lim ? p1 : 0.f);
-            }
-          } else {
-            pp = ptx::f2_pack(ptx::ex2(a0), ptx::ex2(a1));
-          }
+          const uint64_t pp = ptx::f2_pack(ptx::ex2(a0), ptx::ex2(a1));
           sp2[(i >> 1) & 3] = ptx::f2_add(sp2[(i >> 1) & 3], pp);
           float p0, p1;
           ptx::f2_unpack(pp, p0, p1);
@@ -566,7 +554,8 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (!ok || n == 0) continue;
       gt += n;
-      if (!__all_sync(0xffffffffu, wait_bar2(&bars->pv_done[t], (uint32_t)((gt - 1) & 1), abort_flag, pb.err))) {
+      // one pv_done phase per unit of this tile (committed after its last PV)
+      if (!__all_sync(0xffffffffu, wait_bar2(&bars->pv_done[t], (uint32_t)(ep & 1), abort_flag, pb.err))) {
         ok = false;
         break;
       }
@@ -593,6 +582,7 @@ __global__ void __launch_bounds__(384, 1)
       // O has been read: the next unit's first PV may overwrite it
       ptx::tc_fence_before();
       ptx::mbar_arrive(&bars->o_free[t]);
+      ++ep;
       if (store && pb.lse != nullptr) pb.lse[(size_t)(w.tile.q_start + rn) * pb.hq + w.h] = (m + log2f(l)) * kLn2;
     }
   }
