@@ -176,8 +176,16 @@ enum {
                                       (default 64; <= 0 restores it) */
   RPA_OPT_FORCE_GENERIC = 1,       /* 1: run every sequence on the generic
                                       kernel (default 0) */
-  RPA_OPT_DISABLE_PREFILL_TC = 2   /* 1: prefill sequences use the generic
+  RPA_OPT_DISABLE_PREFILL_TC = 2,  /* 1: prefill sequences use the generic
                                       kernel instead of tensor cores */
+  RPA_OPT_PREFILL_SMS = 3,         /* SMs given to the prefill kernel when
+                                      RPA_OPT_CONCURRENT_MIXED is on (0 =
+                                      chosen from the batch's estimated FLOPs
+                                      and bytes) */
+  RPA_OPT_CONCURRENT_MIXED = 4     /* 1: run the prefill and decode work of a
+                                      mixed batch concurrently on two streams
+                                      (default 0: one after the other, faster
+                                      on the measured mixes) */
 };
 RPA_API int64_t rpa_set_option(int32_t option, int64_t value);
 

@@ -26,6 +26,8 @@ RPA_DEV_TIMEOUT = 0x2
 RPA_OPT_DECODE_CHUNK_BLOCKS = 0
 RPA_OPT_FORCE_GENERIC = 1
 RPA_OPT_DISABLE_PREFILL_TC = 2
+RPA_OPT_PREFILL_SMS = 3
+RPA_OPT_CONCURRENT_MIXED = 4
 
 
 class rpa_dims(ctypes.Structure):

@@ -87,6 +87,14 @@ __device__ __forceinline__ void setmaxnreg_dec96() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 96;" ::: "memory");
 }
 
+// Unit order of a persistent CTA: round r takes unit r * G + b on even
+// rounds and r * G + (G - 1 - b) on odd ones ("snake"), so that with the
+// units sorted heaviest first every CTA gets a similar share of the work.
+__device__ __forceinline__ int unit_of(int r) {
+  const int G = gridDim.x, b = blockIdx.x;
+  return r * G + ((r & 1) ? G - 1 - b : b);
+}
+
 // Geometry of one work unit (a 256-row item of one sequence, one query head).
 struct Unit {
   PrefillTile tile;
@@ -179,7 +187,7 @@ __device__ __forceinline__ void mma_loop(Bars2 *bars, volatile int *abort_flag, 
   uint32_t *err = pb.err;
   int g0 = 0, gt0 = 0, gt1 = 0, ep0 = 0, ep1 = 0, uq = 0;
   bool ok = true;
-  for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x, ++uq) {
+  for (int r = 0, u = unit_of(0); ok && u < n_units; u = unit_of(++r), ++uq) {
     const Unit w = make_unit<BM, BN>(tiles, u, pb);
     const int n0 = w.n_t[0], n1 = w.n_t[1], nb = w.nb;
     ok = wait_all(&bars->q_full, (uint32_t)(uq & 1), abort_flag, err);
@@ -233,9 +241,10 @@ __device__ __forceinline__ void mma_loop(Bars2 *bars, volatile int *abort_flag, 
   __syncwarp();
 }
 
-// Persistent: CTA b handles units b, b + gridDim.x, ... of the list of
-// (item, query head) units; items are sorted heaviest first on the host and
-// the heads of one item are consecutive (their K/V blocks are shared in L2).
+// Persistent: each CTA walks its units in the order of unit_of() over the
+// list of (item, query head) units; items are sorted heaviest first on the
+// host and the heads of one item are consecutive (their K/V blocks are
+// shared in L2).
 // Every barrier parity runs on counters that span units, so the producer
 // loads the next unit's Q and K/V while the current one finishes and the MMA
 // warp starts the next unit while the softmax warps are still storing O.
@@ -307,7 +316,7 @@ __global__ void __launch_bounds__(384, 1)
       int g = 0;            // K/V blocks queued so far (all units)
       int uq = 0;           // units started
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x, ++uq) {
+      for (int r = 0, u = unit_of(0); ok && u < n_units; u = unit_of(++r), ++uq) {
         const Unit w = make_unit<BM, BN>(tiles, u, pb);
         const int32_t *pt_row = pb.page_table + (size_t)w.tile.seq * pb.max_pages;
         // Q of both tiles, once the previous unit's QK MMAs are done with sQ
@@ -429,7 +438,7 @@ __global__ void __launch_bounds__(384, 1)
       const __nv_bfloat16 *vn = reinterpret_cast<const __nv_bfloat16 *>(pb.v_new);
       __nv_bfloat16 *kc = reinterpret_cast<__nv_bfloat16 *>(pb.k_cache);
       __nv_bfloat16 *vc = reinterpret_cast<__nv_bfloat16 *>(pb.v_cache);
-      for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+      for (int r = 0, u = unit_of(0); u < n_units; u = unit_of(++r)) {
         const Unit w = make_unit<BM, BN>(tiles, u, pb);
         const int32_t *pt_row = pb.page_table + (size_t)w.tile.seq * pb.max_pages;
         const int gidx = w.h % G;
@@ -461,7 +470,7 @@ __global__ void __launch_bounds__(384, 1)
     int gt = 0;                                  // blocks of this tile consumed so far
     int ep = 0;                                  // units in which this tile had rows
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+    for (int r = 0, u = unit_of(0); ok && u < n_units; u = unit_of(++r)) {
       const Unit w = make_unit<BM, BN>(tiles, u, pb);
       const int n = w.n_t[t];
       const int rn = w.r0 + t * BM + row;        // new-token index of this row
@@ -594,7 +603,7 @@ __global__ void __launch_bounds__(384, 1)
 }
 
 template <int D>
-cudaError_t launch_t(const Problem &pb, const PrefillTile *tiles, int n_tiles, cudaStream_t stream) {
+cudaError_t launch_t(const Problem &pb, const PrefillTile *tiles, int n_tiles, int max_ctas, cudaStream_t stream) {
   using S = P2Shape<D>;
   CUtensorMap tq, tkc, tvc, tkn, tvn;
   const uint64_t qdims[3] = {(uint64_t)D, (uint64_t)pb.hq, (uint64_t)pb.total_q};
@@ -623,18 +632,20 @@ cudaError_t launch_t(const Problem &pb, const PrefillTile *tiles, int n_tiles, c
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
       sms = 148;
   }
-  const int grid = n_units < sms ? n_units : sms;
+  int grid = n_units < sms ? n_units : sms;
+  if (max_ctas > 0 && grid > max_ctas) grid = max_ctas;
   kern<<<grid, 384, S::kSmem, stream>>>(tq, tkc, tvc, tkn, tvn, pb, tiles, n_units, pb.scale * kLog2e);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_prefill2(const Problem &pb, const PrefillTile *tiles, int n_tiles, cudaStream_t stream) {
+cudaError_t launch_prefill2(const Problem &pb, const PrefillTile *tiles, int n_tiles, int max_ctas,
+                            cudaStream_t stream) {
   if (n_tiles <= 0) return cudaSuccess;
   switch (pb.d) {
-    case 64: return launch_t<64>(pb, tiles, n_tiles, stream);
-    case 128: return launch_t<128>(pb, tiles, n_tiles, stream);
+    case 64: return launch_t<64>(pb, tiles, n_tiles, max_ctas, stream);
+    case 128: return launch_t<128>(pb, tiles, n_tiles, max_ctas, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -18,8 +18,10 @@
 //              valid key (past the context, past the sequence, bad pages)
 //              are zeroed before the block is released, so stale or NaN
 //              slots never reach the tensor cores.
-//   warp 5     TMEM owner and MMA issuer (one thread): S = Q K^T into one of
-//              two TMEM buffers, then O += P V with P read from TMEM.
+//   warp 5     TMEM owner and MMA issue (all lanes run the loop, one elected
+//              lane issues): S = Q K^T into one of two TMEM buffers, then
+//              O += P V with P read from TMEM.  The producer warp issues its
+//              copies the same way.
 //
 // Keys are ordered as context blocks [0, c) followed by new-token blocks
 // starting at c, so with BN = 128 the causal diagonal of a 128-row tile is
@@ -79,6 +81,11 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
     }
   }
   return true;
+}
+
+// wait_bar by every lane of a warp, with a warp-uniform result.
+__device__ __forceinline__ bool wait_all1(uint64_t *bar, uint32_t parity, volatile int *abort_flag, uint32_t *err) {
+  return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_flag, err));
 }
 
 template <int D>
@@ -150,11 +157,9 @@ __global__ void __launch_bounds__(192, 1)
     const int nseg = BN / br;                  // <= 16
     uint32_t fix_phase = 0;
     int issued = 0;                            // blocks whose copies were queued
-    if (lane == 0) {
-      ptx::mbar_arrive_expect_tx(&bars->q_full, S::kQBytes);
-      for (int hh = 0; hh < S::kHalves; ++hh)
-        ptx::tma_load_3d(sQ + hh * BM * 128, &tm_q, &bars->q_full, hh * 64, h, tile.q_start + r0);
-    }
+    ptx::mbar_arrive_expect_tx_elect(&bars->q_full, S::kQBytes);
+    for (int hh = 0; hh < S::kHalves; ++hh)
+      ptx::tma_load_3d_elect(sQ + hh * BM * 128, &tm_q, &bars->q_full, hh * 64, h, tile.q_start + r0);
     for (int j = 0; j < nb; ++j) {
       const int s = j % NS;
       const uint32_t ph = (uint32_t)((j / NS) & 1);
@@ -185,39 +190,33 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t blk_bytes = ctx ? (uint32_t)__popc(loaded_mask) * seg_bytes : (uint32_t)S::kKVBytes;
 
       if (j >= NS) {
-        if (!wait_bar(&bars->k_empty[s], ph ^ 1u, abort_flag, pb.err)) break;
-        if (!wait_bar(&bars->v_empty[s], ph ^ 1u, abort_flag, pb.err)) break;
+        if (!wait_all1(&bars->k_empty[s], ph ^ 1u, abort_flag, pb.err)) break;
+        if (!wait_all1(&bars->v_empty[s], ph ^ 1u, abort_flag, pb.err)) break;
       }
-      if (lane == 0) {
-        uint64_t *kb = fix ? &bars->fix : &bars->k_full[s];
-        uint64_t *vb = fix ? &bars->fix : &bars->v_full[s];
-        if (fix) {
-          ptx::mbar_arrive_expect_tx(&bars->fix, 2 * blk_bytes);
-        } else {
-          ptx::mbar_arrive_expect_tx(&bars->k_full[s], blk_bytes);
-          ptx::mbar_arrive_expect_tx(&bars->v_full[s], blk_bytes);
-        }
-        if (!ctx) {
-          const int row = tile.q_start + pos0;
-          for (int hh = 0; hh < S::kHalves; ++hh) {
-            ptx::tma_load_3d(dk + hh * BN * 128, &tm_kn, kb, hh * 64, hk, row);
-            ptx::tma_load_3d(dv + hh * BN * 128, &tm_vn, vb, hh * 64, hk, row);
-          }
-        }
+      uint64_t *kb = fix ? &bars->fix : &bars->k_full[s];
+      uint64_t *vb = fix ? &bars->fix : &bars->v_full[s];
+      if (fix) {
+        ptx::mbar_arrive_expect_tx_elect(&bars->fix, 2 * blk_bytes);
+      } else {
+        ptx::mbar_arrive_expect_tx_elect(&bars->k_full[s], blk_bytes);
+        ptx::mbar_arrive_expect_tx_elect(&bars->v_full[s], blk_bytes);
       }
-      if (ctx) {
-        // every lane takes part in the broadcast of segment sg's page id;
-        // lane 0 queues the copies
+      if (!ctx) {
+        const int row = tile.q_start + pos0;
+        for (int hh = 0; hh < S::kHalves; ++hh) {
+          ptx::tma_load_3d_elect(dk + hh * BN * 128, &tm_kn, kb, hh * 64, hk, row);
+          ptx::tma_load_3d_elect(dv + hh * BN * 128, &tm_vn, vb, hh * 64, hk, row);
+        }
+      } else {
+        // every lane takes part in the broadcast of segment sg's page id
         for (int sg = 0; sg < nseg; ++sg) {
           const int pg = __shfl_sync(0xffffffffu, page, sg);
-          if (lane != 0 || !((loaded_mask >> sg) & 1u)) continue;
-          uint64_t *kb = fix ? &bars->fix : &bars->k_full[s];
-          uint64_t *vb = fix ? &bars->fix : &bars->v_full[s];
+          if (!((loaded_mask >> sg) & 1u)) continue;
           const int sp = pos0 + sg * br;
           const int row = pg * pb.p + (sp % pb.p);
           for (int hh = 0; hh < S::kHalves; ++hh) {
-            ptx::tma_load_3d(dk + hh * BN * 128 + sg * br * 128, &tm_kc, kb, hh * 64, hk, row);
-            ptx::tma_load_3d(dv + hh * BN * 128 + sg * br * 128, &tm_vc, vb, hh * 64, hk, row);
+            ptx::tma_load_3d_elect(dk + hh * BN * 128 + sg * br * 128, &tm_kc, kb, hh * 64, hk, row);
+            ptx::tma_load_3d_elect(dv + hh * BN * 128 + sg * br * 128, &tm_vc, vb, hh * 64, hk, row);
           }
         }
       }
@@ -226,7 +225,7 @@ __global__ void __launch_bounds__(192, 1)
         // Wait for this block's copies (the private barrier completes even
         // with no copies: the arrival carried zero expected bytes), zero
         // every row that holds no valid key, then publish the block.
-        const bool ok = wait_bar(&bars->fix, fix_phase, abort_flag, pb.err);
+        const bool ok = wait_all1(&bars->fix, fix_phase, abort_flag, pb.err);
         fix_phase ^= 1u;
         if (!ok) break;
         for (int r = lane; r < BN; r += 32) {
@@ -244,10 +243,8 @@ __global__ void __launch_bounds__(192, 1)
         }
         ptx::fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) {
-          ptx::mbar_arrive(&bars->k_full[s]);
-          ptx::mbar_arrive(&bars->v_full[s]);
-        }
+        ptx::mbar_arrive_elect(&bars->k_full[s]);
+        ptx::mbar_arrive_elect(&bars->v_full[s]);
       }
     }
     // Before the CTA can end, every copy this warp queued must have landed
@@ -262,57 +259,59 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
   } else if (warp == 5) {
     // ---------------------------------------------------------------- MMA
-    if (lane == 0) {
+    // All 32 lanes run the loop; one elected lane issues each MMA / commit.
+    {
       const uint32_t tS[2] = {tmem + S::kColS0, tmem + S::kColS1};
       const uint32_t tO = tmem + S::kColO;
       constexpr uint32_t idesc_qk = ptx::umma_idesc_bf16(128, BN, false);
       constexpr uint32_t idesc_pv = ptx::umma_idesc_bf16(128, D, true);
-      const uint32_t q_addr = ptx::smem_u32(sQ);
-      const uint32_t k_addr = ptx::smem_u32(sK);
-      const uint32_t v_addr = ptx::smem_u32(sV);
-      bool ok = wait_bar(&bars->q_full, 0, abort_flag, pb.err);
+      const uint64_t dq0 = ptx::umma_desc_sw128(ptx::smem_u32(sQ), 16, 1024);
+      const uint64_t dk0 = ptx::umma_desc_sw128(ptx::smem_u32(sK), 16, 1024);
+      const uint64_t dv0 = ptx::umma_desc_sw128(ptx::smem_u32(sV), BN * 128, 1024);
+      bool ok = wait_all1(&bars->q_full, 0, abort_flag, pb.err);
       auto pv = [&](int i) -> bool {
         const int b = i & 1, s = i % NS;
-        if (!wait_bar(&bars->p_full[b], (uint32_t)((i >> 1) & 1), abort_flag, pb.err)) return false;
-        if (!wait_bar(&bars->v_full[s], (uint32_t)((i / NS) & 1), abort_flag, pb.err)) return false;
+        if (!wait_all1(&bars->p_full[b], (uint32_t)((i >> 1) & 1), abort_flag, pb.err)) return false;
+        if (!wait_all1(&bars->v_full[s], (uint32_t)((i / NS) & 1), abort_flag, pb.err)) return false;
         ptx::tc_fence_after();
+        const uint64_t dv = dv0 + (uint64_t)((s * S::kKVBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bdesc = ptx::umma_desc_sw128(v_addr + s * S::kKVBytes + kk * 16 * 128, BN * 128, 1024);
-          ptx::umma_ts(tO, tS[b] + kk * 8, bdesc, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
-        }
-        ptx::umma_commit(&bars->pv_done[b]);
-        ptx::umma_commit(&bars->v_empty[s]);
+        for (int kk = 0; kk < BN / 16; ++kk)
+          ptx::umma_ts_elect(tO, tS[b] + kk * 8, dv + (uint64_t)((kk * 16 * 128) >> 4), idesc_pv,
+                             (i > 0 || kk > 0) ? 1u : 0u);
+        ptx::umma_commit_elect(&bars->pv_done[b]);
+        ptx::umma_commit_elect(&bars->v_empty[s]);
         return true;
       };
       for (int j = 0; ok && j < nb; ++j) {
         const int b = j & 1, s = j % NS;
-        if (j >= 2 && !wait_bar(&bars->pv_done[b], (uint32_t)(((j - 2) >> 1) & 1), abort_flag, pb.err)) {
+        if (j >= 2 && !wait_all1(&bars->pv_done[b], (uint32_t)(((j - 2) >> 1) & 1), abort_flag, pb.err)) {
           ok = false;
           break;
         }
-        if (!wait_bar(&bars->k_full[s], (uint32_t)((j / NS) & 1), abort_flag, pb.err)) {
+        if (!wait_all1(&bars->k_full[s], (uint32_t)((j / NS) & 1), abort_flag, pb.err)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
+        const uint64_t dk = dk0 + (uint64_t)((s * S::kKVBytes) >> 4);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t off = (ks & 3) * 32;   // 16 bf16 = 32 bytes inside a 128-byte row
-          const uint64_t adesc = ptx::umma_desc_sw128(q_addr + (ks >> 2) * BM * 128 + off, 16, 1024);
-          const uint64_t bdesc = ptx::umma_desc_sw128(k_addr + s * S::kKVBytes + (ks >> 2) * BN * 128 + off, 16, 1024);
-          ptx::umma_ss(tS[b], adesc, bdesc, idesc_qk, ks > 0 ? 1u : 0u);
+          // 16 bf16 = 32 bytes inside a 128-byte row; 64-column tiles apart
+          const uint32_t offq = ((ks >> 2) * BM * 128 + (ks & 3) * 32) >> 4;
+          const uint32_t offk = ((ks >> 2) * BN * 128 + (ks & 3) * 32) >> 4;
+          ptx::umma_ss_elect(tS[b], dq0 + offq, dk + offk, idesc_qk, ks > 0 ? 1u : 0u);
         }
-        ptx::umma_commit(&bars->s_full[b]);
-        ptx::umma_commit(&bars->k_empty[s]);
+        ptx::umma_commit_elect(&bars->s_full[b]);
+        ptx::umma_commit_elect(&bars->k_empty[s]);
         if (j >= 1 && !pv(j - 1)) {
           ok = false;
           break;
         }
       }
       if (ok) pv(nb - 1);
-      // drain: wait until every MMA this thread issued has completed
-      ptx::umma_commit(&bars->drain);
+      // drain: wait until every MMA of this CTA has completed
+      ptx::umma_commit_elect(&bars->drain);
       ptx::mbar_wait(&bars->drain, 0);
     }
     __syncwarp();

@@ -27,6 +27,8 @@ namespace {
 std::atomic<int64_t> g_opt_decode_chunk{0};
 std::atomic<int64_t> g_opt_force_generic{0};
 std::atomic<int64_t> g_opt_disable_prefill_tc{0};
+std::atomic<int64_t> g_opt_prefill_sms{0};
+std::atomic<int64_t> g_opt_concurrent_mixed{0};
 
 constexpr int kDefaultDecodeChunkBlocks = 64;
 // 256 blocks of 16 tokens touch at most 4096 / 8 + 1 pages, within the decode
@@ -100,6 +102,8 @@ struct HostPlan {
   int32_t n_partials = 0;
   int32_t decode_max_splits = 0;
   int32_t num_decode = 0, num_prefill = 0, num_generic = 0, num_empty = 0;
+  double decode_bytes = 0.0;     // K/V bytes the decode kernel streams
+  double prefill_flops = 0.0;    // visible (q, k) pairs x 4 D Hq
   PlanLayout layout{};
 };
 
@@ -131,6 +135,7 @@ void build_plan(const int32_t *cu, const int32_t *kv, int32_t n, const int32_t *
       }
       case kDecode: {
         ++hp.num_decode;
+        hp.decode_bytes += (double)kvl * d->num_kv_heads * d->head_dim * 4.0;
         const int32_t nblk = (kvl + kDecodeBlock - 1) / kDecodeBlock;
         const int32_t nsplit = (int32_t)((nblk + chunk - 1) / chunk);
         const int32_t per = (nblk + nsplit - 1) / nsplit;
@@ -160,6 +165,10 @@ void build_plan(const int32_t *cu, const int32_t *kv, int32_t n, const int32_t *
       }
       case kPrefill: {
         ++hp.num_prefill;
+        {
+          const double q = ql, c = (double)kvl - ql;
+          hp.prefill_flops += 4.0 * d->head_dim * d->num_q_heads * q * (c + (q + 1) / 2.0);
+        }
         const int32_t item_rows = prefill_item_rows(d->head_dim);
         for (int32_t r = 0; r < ql; r += item_rows) {
           PrefillTile t{};
@@ -231,6 +240,8 @@ struct Slot {
   float *partial = nullptr;  // o then lse
   int64_t partial_floats = 0;
   cudaEvent_t done = nullptr;
+  cudaEvent_t fork = nullptr;   // caller's stream -> side stream
+  cudaEvent_t join = nullptr;   // side stream -> caller's stream
   bool pending = false;
 };
 
@@ -238,6 +249,8 @@ struct DeviceWs {
   std::mutex mu;
   bool init = false;
   uint32_t *err = nullptr;
+  cudaStream_t side = nullptr;  // prefill of mixed batches runs here
+  int sms = 0;
   Slot slots[kSlots];
   int next = 0;
 };
@@ -249,7 +262,15 @@ int ensure_init(DeviceWs &ws) {
   if (cudaMalloc(&ws.err, sizeof(uint32_t)) != cudaSuccess) return RPA_ERR_OOM;
   if (cudaMemset(ws.err, 0, sizeof(uint32_t)) != cudaSuccess) return RPA_ERR_CUDA;
   for (auto &s : ws.slots)
-    if (cudaEventCreateWithFlags(&s.done, cudaEventDisableTiming) != cudaSuccess) return RPA_ERR_CUDA;
+    if (cudaEventCreateWithFlags(&s.done, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming) != cudaSuccess)
+      return RPA_ERR_CUDA;
+  if (cudaStreamCreateWithFlags(&ws.side, cudaStreamNonBlocking) != cudaSuccess) return RPA_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&ws.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || ws.sms <= 0)
+    ws.sms = 148;
   ws.init = true;
   return RPA_OK;
 }
@@ -354,6 +375,8 @@ extern "C" RPA_API int64_t rpa_set_option(int32_t option, int64_t value) {
     case RPA_OPT_DECODE_CHUNK_BLOCKS: return g_opt_decode_chunk.exchange(value);
     case RPA_OPT_FORCE_GENERIC: return g_opt_force_generic.exchange(value);
     case RPA_OPT_DISABLE_PREFILL_TC: return g_opt_disable_prefill_tc.exchange(value);
+    case RPA_OPT_PREFILL_SMS: return g_opt_prefill_sms.exchange(value);
+    case RPA_OPT_CONCURRENT_MIXED: return g_opt_concurrent_mixed.exchange(value);
     default: return -1;
   }
 }
@@ -439,12 +462,34 @@ extern "C" RPA_API int rpa_forward(const void *q, const void *k_new, const void 
     float *partial_o = slot.partial;
     float *partial_lse = slot.partial ? slot.partial + L.n_partials * dims->num_kv_heads * G * dims->head_dim : nullptr;
     cudaError_t e = cudaSuccess;
+    // Optionally, a batch with both prefill and decode work runs them
+    // concurrently: the compute-bound prefill kernel on the side stream with a
+    // share of the SMs, the bandwidth-bound decode kernel on the caller's
+    // stream on the rest.
+    const bool mixed = L.n_prefill_tiles > 0 && (L.n_decode_items > 0 || L.n_generic_rows > 0) &&
+                       g_opt_concurrent_mixed.load() != 0;
+    cudaStream_t pstream = stream;
+    int prefill_ctas = 0;
+    if (mixed) {
+      int64_t k = g_opt_prefill_sms.load();
+      if (k <= 0) {
+        // balance the two finishing times: prefill at ~0.9 PFLOP/s and decode
+        // at ~5.5 TB/s when each has the whole GPU
+        const double tp = hp.prefill_flops / 0.9e15, td = hp.decode_bytes / 5.5e12;
+        k = (int64_t)(ws.sms * (tp / (tp + td + 1e-30)) + 0.5);
+      }
+      prefill_ctas = (int)std::max<int64_t>(8, std::min<int64_t>(k, ws.sms - 8));
+      pstream = ws.side;
+      if (cudaEventRecord(slot.fork, stream) != cudaSuccess || cudaStreamWaitEvent(pstream, slot.fork, 0) != cudaSuccess)
+        return RPA_ERR_CUDA;
+    }
     if (L.n_prefill_tiles > 0 && e == cudaSuccess)
-      e = traced(RPA_KERNEL_PREFILL, stream, [&] {
+      e = traced(RPA_KERNEL_PREFILL, pstream, [&] {
         const PrefillTile *tiles = (const PrefillTile *)(slot.dev + L.prefill_off);
-        return pb.d <= 128 ? launch_prefill2(pb, tiles, (int)L.n_prefill_tiles, stream)
-                           : launch_prefill(pb, tiles, (int)L.n_prefill_tiles, stream);
+        return pb.d <= 128 ? launch_prefill2(pb, tiles, (int)L.n_prefill_tiles, prefill_ctas, pstream)
+                           : launch_prefill(pb, tiles, (int)L.n_prefill_tiles, pstream);
       });
+    if (mixed && cudaEventRecord(slot.join, pstream) != cudaSuccess) e = cudaErrorUnknown;
     if (L.n_decode_items > 0 && e == cudaSuccess)
       e = traced(RPA_KERNEL_DECODE, stream, [&] {
         return launch_decode(pb, (const DecodeItem *)(slot.dev + L.decode_off),
@@ -460,6 +505,9 @@ extern "C" RPA_API int rpa_forward(const void *q, const void *k_new, const void 
         return launch_generic(pb, (const GenericSeq *)(slot.dev + L.generic_off),
                               (int)L.n_generic_seqs, (int)L.n_generic_rows, stream);
       });
+    // join: the caller's stream waits for the side stream (also on errors,
+    // so that nothing of this call is left running unordered)
+    if (mixed && cudaStreamWaitEvent(stream, slot.join, 0) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;
     if (cudaEventRecord(slot.done, stream) == cudaSuccess) slot.pending = true;
     return e == cudaSuccess ? RPA_OK : RPA_ERR_CUDA;
   } catch (const std::bad_alloc &) {
