@@ -111,7 +111,7 @@ extern "C" RPA_API int rpa_decode_noalloc(const void *q, const void *k_new, cons
   }
   unsigned char *scratch = static_cast<unsigned char *>(g_scratch_ptr[dev]);
 
-  // ---- plan: the same chunking as rpa_forward's decode work list
+  // ---- plan: near-equal chunks of at most kChunkBlocks 16-token blocks per sequence
   int32_t ni = 0, nc = 0, np = 0;
   for (int32_t s = 0; s < num_seqs; ++s) {
     const int32_t kvl = kv_lens[s];

@@ -79,6 +79,37 @@ def test_without_distribution_and_shuffled_order(oracle_mod):
     full_check(oracle_mod, prob, use_distribution=False)
 
 
+def test_concurrent_mixed_batch(oracle_mod):
+    """The opt-in concurrent execution of a mixed batch (prefill on a second
+    stream with a share of the SMs, decode on the caller's stream) gives the
+    oracle's results too."""
+    from ragged_paged_attention_03_b200 import binding
+    old_c = binding.rpa_set_option(binding.RPA_OPT_CONCURRENT_MIXED, 1)
+    old_k = binding.rpa_set_option(binding.RPA_OPT_PREFILL_SMS, 20)
+    try:
+        prob = I.make_problem([1] * 6 + [300, 77], [40, 900, 2100, 1, 17, 300, 300, 500],
+                              num_q_heads=32, num_kv_heads=8, head_dim=128, page_size=16,
+                              dtype=I.BF16, seed=21, pool=1.3)
+        full_check(oracle_mod, prob)
+    finally:
+        binding.rpa_set_option(binding.RPA_OPT_CONCURRENT_MIXED, old_c)
+        binding.rpa_set_option(binding.RPA_OPT_PREFILL_SMS, old_k)
+
+
+@pytest.mark.parametrize("chunk", [1, 3])
+def test_decode_heavy_split_kv(oracle_mod, chunk):
+    """Decode sequences cut into many small work items (1 or 3 blocks of 16
+    tokens each) merged by the log-sum-exp combine."""
+    from ragged_paged_attention_03_b200 import binding
+    old = binding.rpa_set_option(binding.RPA_OPT_DECODE_CHUNK_BLOCKS, chunk)
+    try:
+        prob = I.make_problem([1] * 5, [1, 16, 33, 500, 1000], num_q_heads=16, num_kv_heads=2,
+                              head_dim=128, page_size=8, dtype=I.BF16, seed=22, pool=1.3)
+        full_check(oracle_mod, prob)
+    finally:
+        binding.rpa_set_option(binding.RPA_OPT_DECODE_CHUNK_BLOCKS, old)
+
+
 def test_bad_page_is_flagged_not_read(oracle_mod):
     """A page-table entry outside the pool is reported through the device
     error word; the kernels never dereference it."""
