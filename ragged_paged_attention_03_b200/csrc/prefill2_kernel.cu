@@ -43,11 +43,14 @@ template <int D>
 struct P2Shape {
   static constexpr int BM = 128;     // rows per tile, two tiles per CTA
   static constexpr int BN = 128;     // keys per block
-  static constexpr int NS = D == 64 ? 3 : 2;
+  // K and V have rings of their own: a K stage is released two MMA groups
+  // before the V stage of the same block, and the next block needs K first.
+  static constexpr int NSK = D == 64 ? 4 : 3;
+  static constexpr int NSV = D == 64 ? 4 : 2;
   static constexpr int kHalves = D / 64;
   static constexpr int kQBytes = kHalves * BM * 128;
   static constexpr int kKVBytes = kHalves * BN * 128;
-  static constexpr int kData = 2 * kQBytes + 2 * NS * kKVBytes;
+  static constexpr int kData = 2 * kQBytes + (NSK + NSV) * kKVBytes;
   static constexpr int kSmem = 1024 + kData + 512;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColO = 256;   // O of tile t at kColO + t * D
@@ -55,7 +58,7 @@ struct P2Shape {
 
 struct Bars2 {
   uint64_t q_full, q_empty;
-  uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
+  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
   uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];
   uint64_t fix, drain;
 };
@@ -122,14 +125,14 @@ __device__ __forceinline__ Unit make_unit(const PrefillTile *tiles, int u, const
   return w;
 }
 
-// QK(t, gblk): S of tile t = Q_t K^T for K/V block gblk (stage gblk % NS).
+// QK(t, gblk): S of tile t = Q_t K^T for K/V block gblk (K stage gblk % NSK).
 template <int D>
 __device__ __forceinline__ bool issue_qk(Bars2 *bars, volatile int *abort_flag, uint32_t *err, uint32_t tS,
                                          uint64_t dq, uint64_t dk0, int gblk, bool wait_k) {
   using S = P2Shape<D>;
   constexpr uint32_t idesc = ptx::umma_idesc_bf16(128, S::BN, false);
-  const int s = gblk % S::NS;
-  if (wait_k && !wait_all(&bars->k_full[s], (uint32_t)((gblk / S::NS) & 1), abort_flag, err)) return false;
+  const int s = gblk % S::NSK;
+  if (wait_k && !wait_all(&bars->k_full[s], (uint32_t)((gblk / S::NSK) & 1), abort_flag, err)) return false;
   ptx::tc_fence_after();
   const uint64_t dk = dk0 + (uint64_t)((s * S::kKVBytes) >> 4);
 #pragma unroll
@@ -148,9 +151,9 @@ __device__ __forceinline__ bool issue_pv(Bars2 *bars, volatile int *abort_flag, 
                                          bool first, bool wait_v) {
   using S = P2Shape<D>;
   constexpr uint32_t idesc = ptx::umma_idesc_bf16(128, D, true);
-  const int s = gblk % S::NS;
+  const int s = gblk % S::NSV;
   if (!wait_all(&bars->p_full[t], (uint32_t)(tblk & 1), abort_flag, err)) return false;
-  if (wait_v && !wait_all(&bars->v_full[s], (uint32_t)((gblk / S::NS) & 1), abort_flag, err)) return false;
+  if (wait_v && !wait_all(&bars->v_full[s], (uint32_t)((gblk / S::NSV) & 1), abort_flag, err)) return false;
   ptx::tc_fence_after();
   const uint64_t dv = dv0 + (uint64_t)((s * S::kKVBytes) >> 4);
 #pragma unroll
@@ -174,7 +177,7 @@ __device__ __forceinline__ void mma_loop(Bars2 *bars, volatile int *abort_flag, 
                                          const PrefillTile *tiles, int n_units, uint32_t tmem, uint32_t q_addr,
                                          uint32_t k_addr, uint32_t v_addr) {
   using S = P2Shape<D>;
-  constexpr int BM = S::BM, BN = S::BN, NS = S::NS;
+  constexpr int BM = S::BM, BN = S::BN, NSK = S::NSK, NSV = S::NSV;
   const uint32_t tS0 = tmem, tS1 = tmem + 128;
   const uint32_t tO0 = tmem + S::kColO, tO1 = tmem + S::kColO + D;
   // Descriptors of the stage-0 / tile-0 operands; the start-address field
@@ -196,7 +199,7 @@ __device__ __forceinline__ void mma_loop(Bars2 *bars, volatile int *abort_flag, 
     if (ok && n0 > 0) ptx::umma_commit_elect(&bars->s_full[0]);
     if (ok && n1 > 0) ok = issue_qk<D>(bars, abort_flag, err, tS1, dq1, dk0, g0, n0 == 0);
     if (ok && n1 > 0) ptx::umma_commit_elect(&bars->s_full[1]);
-    if (ok) ptx::umma_commit_elect(&bars->k_empty[g0 % NS]);
+    if (ok) ptx::umma_commit_elect(&bars->k_empty[g0 % NSK]);
     if (ok && nb == 1) ptx::umma_commit_elect(&bars->q_empty);
     if (ok && n0 > 0) {
       // O_0 is overwritten by the unit's first PV: the softmax warps must
@@ -218,12 +221,12 @@ __device__ __forceinline__ void mma_loop(Bars2 *bars, volatile int *abort_flag, 
         if (ok) ok = issue_pv<D>(bars, abort_flag, err, 1, tS1, tO1, dv0, g0 + j, gt1 + j, j == 0, j >= n0);
         if (ok && j + 1 == n1) ptx::umma_commit_elect(&bars->pv_done[1]);
       }
-      if (ok) ptx::umma_commit_elect(&bars->v_empty[(g0 + j) % NS]);   // both PVs of block j issued
+      if (ok) ptx::umma_commit_elect(&bars->v_empty[(g0 + j) % NSV]);   // both PVs of block j issued
       if (ok && j + 1 < n1) {
         ok = issue_qk<D>(bars, abort_flag, err, tS1, dq1, dk0, g0 + j + 1, !k_next_waited);
         if (ok) ptx::umma_commit_elect(&bars->s_full[1]);
       }
-      if (ok && j + 1 < nb) ptx::umma_commit_elect(&bars->k_empty[(g0 + j + 1) % NS]);
+      if (ok && j + 1 < nb) ptx::umma_commit_elect(&bars->k_empty[(g0 + j + 1) % NSK]);
       if (ok && j + 2 == nb) ptx::umma_commit_elect(&bars->q_empty);   // last QK of the unit issued
       if (ok && j + 1 < n0) {
         ok = issue_pv<D>(bars, abort_flag, err, 0, tS0, tO0, dv0, g0 + j + 1, gt0 + j + 1, false, true);
@@ -255,12 +258,12 @@ __global__ void __launch_bounds__(384, 1)
                     const __grid_constant__ CUtensorMap tm_vn, const Problem pb,
                     const PrefillTile *__restrict__ tiles, int n_units, float scale_log2) {
   using S = P2Shape<D>;
-  constexpr int BM = S::BM, BN = S::BN, NS = S::NS;
+  constexpr int BM = S::BM, BN = S::BN, NSK = S::NSK, NSV = S::NSV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sQ = base;                              // tile t at sQ + t * kQBytes
   uint8_t *sK = sQ + 2 * S::kQBytes;
-  uint8_t *sV = sK + NS * S::kKVBytes;
+  uint8_t *sV = sK + NSK * S::kKVBytes;
   Bars2 *bars = reinterpret_cast<Bars2 *>(base + S::kData);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -273,9 +276,11 @@ __global__ void __launch_bounds__(384, 1)
   if (tid == 0) {
     ptx::mbar_init(&bars->q_full, 1);
     ptx::mbar_init(&bars->q_empty, 1);
-    for (int i = 0; i < NS; ++i) {
+    for (int i = 0; i < NSK; ++i) {
       ptx::mbar_init(&bars->k_full[i], 1);
       ptx::mbar_init(&bars->k_empty[i], 1);
+    }
+    for (int i = 0; i < NSV; ++i) {
       ptx::mbar_init(&bars->v_full[i], 1);
       ptx::mbar_init(&bars->v_empty[i], 1);
     }
@@ -313,7 +318,9 @@ __global__ void __launch_bounds__(384, 1)
       const int br = pb.p < BN ? pb.p : BN;
       const int nseg = BN / br;
       uint32_t fix_phase = 0;
-      int g = 0;            // K/V blocks queued so far (all units)
+      int g = 0;            // K/V blocks started so far (all units)
+      int gk = 0, gv = 0;   // blocks whose K (V) copies were queued and published
+      bool fix_pending = false;
       int uq = 0;           // units started
       bool ok = true;
       for (int r = 0, u = unit_of(0); ok && u < n_units; u = unit_of(++r), ++uq) {
@@ -329,10 +336,10 @@ __global__ void __launch_bounds__(384, 1)
                                    w.tile.q_start + w.r0 + t * BM);
         }
         for (int j = 0; j < w.nb; ++j, ++g) {
-          const int s = g % NS;
-          const uint32_t ph = (uint32_t)((g / NS) & 1);
-          uint8_t *dk = sK + s * S::kKVBytes;
-          uint8_t *dv = sV + s * S::kKVBytes;
+          const int sk = g % NSK, sv = g % NSV;
+          const uint32_t phk = (uint32_t)((g / NSK) & 1), phv = (uint32_t)((g / NSV) & 1);
+          uint8_t *dk = sK + sk * S::kKVBytes;
+          uint8_t *dv = sV + sv * S::kKVBytes;
           const bool ctx = j < w.n_ctx;
           const int pos0 = ctx ? j * BN : (j - w.n_ctx) * BN;
           const int valid = min(BN, (ctx ? w.c : w.tile.q_len) - pos0);
@@ -354,76 +361,89 @@ __global__ void __launch_bounds__(384, 1)
           const bool fix = valid < BN || __any_sync(0xffffffffu, seg_bad);
           const uint32_t seg_bytes = (uint32_t)(S::kHalves * br * 128);
           const uint32_t blk_bytes = ctx ? (uint32_t)__popc(loaded_mask) * seg_bytes : (uint32_t)S::kKVBytes;
-          if (g >= NS) {
-            if (!wait_all(&bars->k_empty[s], ph ^ 1u, abort_flag, pb.err) ||
-                !wait_all(&bars->v_empty[s], ph ^ 1u, abort_flag, pb.err)) {
+          // the copies of one operand (K or V) of this block into dst
+          auto load = [&](uint8_t *dst, const CUtensorMap *tm_new, const CUtensorMap *tm_ctx, uint64_t *bar) {
+            if (!ctx) {
+              const int row = w.tile.q_start + pos0;
+              for (int hh = 0; hh < S::kHalves; ++hh)
+                ptx::tma_load_3d_elect(dst + hh * BN * 128, tm_new, bar, hh * 64, w.hk, row);
+            } else {
+              for (int sg = 0; sg < nseg; ++sg) {
+                const int pg = __shfl_sync(0xffffffffu, page, sg);
+                if (!((loaded_mask >> sg) & 1u)) continue;
+                const int sp = pos0 + sg * br;
+                const int row = pg * pb.p + (sp % pb.p);
+                for (int hh = 0; hh < S::kHalves; ++hh)
+                  ptx::tma_load_3d_elect(dst + hh * BN * 128 + sg * br * 128, tm_ctx, bar, hh * 64, w.hk, row);
+              }
+            }
+          };
+          if (!fix) {
+            // K as soon as its stage is free, then V
+            if (g >= NSK && !wait_all(&bars->k_empty[sk], phk ^ 1u, abort_flag, pb.err)) {
               ok = false;
               break;
             }
+            ptx::mbar_arrive_expect_tx_elect(&bars->k_full[sk], blk_bytes);
+            load(dk, &tm_kn, &tm_kc, &bars->k_full[sk]);
+            ++gk;
+            if (g >= NSV && !wait_all(&bars->v_empty[sv], phv ^ 1u, abort_flag, pb.err)) {
+              ok = false;
+              break;
+            }
+            ptx::mbar_arrive_expect_tx_elect(&bars->v_full[sv], blk_bytes);
+            load(dv, &tm_vn, &tm_vc, &bars->v_full[sv]);
+            ++gv;
+            continue;
           }
-          uint64_t *kb = fix ? &bars->fix : &bars->k_full[s];
-          uint64_t *vb = fix ? &bars->fix : &bars->v_full[s];
-          if (fix) {
-            ptx::mbar_arrive_expect_tx_elect(&bars->fix, 2 * blk_bytes);
-          } else {
-            ptx::mbar_arrive_expect_tx_elect(&bars->k_full[s], blk_bytes);
-            ptx::mbar_arrive_expect_tx_elect(&bars->v_full[s], blk_bytes);
+          // Partial block or bad pages: both operands through the private
+          // barrier, then zero the rows without a valid key and publish.
+          if ((g >= NSK && !wait_all(&bars->k_empty[sk], phk ^ 1u, abort_flag, pb.err)) ||
+              (g >= NSV && !wait_all(&bars->v_empty[sv], phv ^ 1u, abort_flag, pb.err))) {
+            ok = false;
+            break;
           }
-          if (!ctx) {
-            const int row = w.tile.q_start + pos0;
+          ptx::mbar_arrive_expect_tx_elect(&bars->fix, 2 * blk_bytes);
+          load(dk, &tm_kn, &tm_kc, &bars->fix);
+          load(dv, &tm_vn, &tm_vc, &bars->fix);
+          // the private barrier completes even when no copy was queued
+          const bool fok = wait_all(&bars->fix, fix_phase, abort_flag, pb.err);
+          fix_phase ^= 1u;
+          if (!fok) {
+            // copies may still be in flight: the drain below waits for them
+            fix_pending = true;
+            ok = false;
+            break;
+          }
+          for (int r = lane; r < BN; r += 32) {
+            const bool bad_row = r >= valid || (ctx && !((loaded_mask >> (r / br)) & 1u));
+            if (!bad_row) continue;
             for (int hh = 0; hh < S::kHalves; ++hh) {
-              ptx::tma_load_3d_elect(dk + hh * BN * 128, &tm_kn, kb, hh * 64, w.hk, row);
-              ptx::tma_load_3d_elect(dv + hh * BN * 128, &tm_vn, vb, hh * 64, w.hk, row);
-            }
-          } else {
-            for (int sg = 0; sg < nseg; ++sg) {
-              const int pg = __shfl_sync(0xffffffffu, page, sg);
-              if (!((loaded_mask >> sg) & 1u)) continue;
-              const int sp = pos0 + sg * br;
-              const int row = pg * pb.p + (sp % pb.p);
-              for (int hh = 0; hh < S::kHalves; ++hh) {
-                ptx::tma_load_3d_elect(dk + hh * BN * 128 + sg * br * 128, &tm_kc, kb, hh * 64, w.hk, row);
-                ptx::tma_load_3d_elect(dv + hh * BN * 128 + sg * br * 128, &tm_vc, vb, hh * 64, w.hk, row);
-              }
-            }
-          }
-          if (fix) {
-            // wait for this block's copies (the private barrier completes
-            // even with none), zero the rows without a valid key, publish
-            const bool fok = wait_all(&bars->fix, fix_phase, abort_flag, pb.err);
-            fix_phase ^= 1u;
-            if (!fok) {
-              ok = false;
-              ++g;
-              break;
-            }
-            for (int r = lane; r < BN; r += 32) {
-              const bool bad_row = r >= valid || (ctx && !((loaded_mask >> (r / br)) & 1u));
-              if (!bad_row) continue;
-              for (int hh = 0; hh < S::kHalves; ++hh) {
-                uint4 *pk = reinterpret_cast<uint4 *>(dk + hh * BN * 128 + r * 128);
-                uint4 *pv = reinterpret_cast<uint4 *>(dv + hh * BN * 128 + r * 128);
+              uint4 *pk = reinterpret_cast<uint4 *>(dk + hh * BN * 128 + r * 128);
+              uint4 *pv = reinterpret_cast<uint4 *>(dv + hh * BN * 128 + r * 128);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                  pk[q] = make_uint4(0, 0, 0, 0);
-                  pv[q] = make_uint4(0, 0, 0, 0);
-                }
+              for (int q = 0; q < 8; ++q) {
+                pk[q] = make_uint4(0, 0, 0, 0);
+                pv[q] = make_uint4(0, 0, 0, 0);
               }
             }
-            ptx::fence_proxy_async_smem();
-            __syncwarp();
-            ptx::mbar_arrive_elect(&bars->k_full[s]);
-            ptx::mbar_arrive_elect(&bars->v_full[s]);
           }
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          ptx::mbar_arrive_elect(&bars->k_full[sk]);
+          ptx::mbar_arrive_elect(&bars->v_full[sv]);
+          ++gk;
+          ++gv;
         }
       }
       // every copy this warp queued must land before the CTA ends
       if (lane == 0) {
         if (uq > 0) ptx::mbar_wait(&bars->q_full, (uint32_t)((uq - 1) & 1));
-        for (int k = g - NS < 0 ? 0 : g - NS; k < g; ++k) {
-          ptx::mbar_wait(&bars->k_full[k % NS], (uint32_t)((k / NS) & 1));
-          ptx::mbar_wait(&bars->v_full[k % NS], (uint32_t)((k / NS) & 1));
-        }
+        for (int k = gk - NSK < 0 ? 0 : gk - NSK; k < gk; ++k)
+          ptx::mbar_wait(&bars->k_full[k % NSK], (uint32_t)((k / NSK) & 1));
+        for (int k = gv - NSV < 0 ? 0 : gv - NSV; k < gv; ++k)
+          ptx::mbar_wait(&bars->v_full[k % NSV], (uint32_t)((k / NSV) & 1));
+        if (fix_pending) ptx::mbar_wait(&bars->fix, fix_phase ^ 1u);
       }
       __syncwarp();
     } else if (warp == 9) {
@@ -472,7 +492,9 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
     for (int r = 0, u = unit_of(0); ok && u < n_units; u = unit_of(++r)) {
       const Unit w = make_unit<BM, BN>(tiles, u, pb);
-      const int n = w.n_t[t];
+      // tile-uniform selects keep the unit in registers (no local memory)
+      const int n = t ? w.n_t[1] : w.n_t[0];
+      const int rows_mine = t ? w.rows_t[1] : w.rows_t[0];
       const int rn = w.r0 + t * BM + row;        // new-token index of this row
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < n; ++j) {
@@ -570,7 +592,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       ptx::tc_fence_after();
       const float inv = 1.f / l;
-      const bool store = row < w.rows_t[t];
+      const bool store = row < rows_mine;
       __nv_bfloat16 *out =
           reinterpret_cast<__nv_bfloat16 *>(pb.out) + ((size_t)(w.tile.q_start + rn) * pb.hq + w.h) * D;
 #pragma unroll
