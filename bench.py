@@ -332,14 +332,26 @@ def cpu_baseline(name, prob_dev, budget_s):
 
 
 # ----------------------------------------------------------------- main
-def dist_setup(args):
+def dist_setup(args, backend="nccl"):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1 and args.impl == "ours":
         import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return world, rank, local
+
+
+def max_over_ranks(x: float, device) -> float:
+    """The largest x over all ranks: each rank runs its own replica, and the
+    slowest one sets the whole job's step time.  Every rank must call it at
+    the same point (it is a collective when more than one rank runs)."""
+    dist = torch.distributed
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 def main():
@@ -414,16 +426,11 @@ def main():
         if i == 0:
             clk = clocks.stop()
         torch.cuda.synchronize(dev)
+        ms = max_over_ranks(ms, dev)
         if world > 1:
-            t = torch.tensor([ms], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            ms = float(t.item())
             torch.distributed.barrier()
         e2e_ms, h2d, d2h = time_e2e(prob, max(10, args.steps // 4), 3, flush, stream)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e2e_ms, dev)
         metric, unit = metric_of(name)
         line = {"metric": metric, "value": value_of(name, work, ms, n), "unit": unit,
                 "ms_per_step": ms,

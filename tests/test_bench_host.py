@@ -1,0 +1,109 @@
+"""Host-side logic of bench.py, on CPU: the multi-rank aggregation (two gloo
+ranks, as torchrun would launch two replicas), the algorithmic work counts
+and the roofline arithmetic.  No GPU and no kernel call."""
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from ragged_paged_attention_03_b200 import inputs as I  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, ms_by_rank, out_q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+
+    class Args:
+        impl = "ours"
+
+    try:
+        got_world, got_rank, _ = bench.dist_setup(Args, backend="gloo")
+        ms = bench.max_over_ranks(ms_by_rank[rank], "cpu")
+        e2e = bench.max_over_ranks(2.0 * ms_by_rank[rank], "cpu")
+        work = {"bytes": 10 ** 9, "flops": 10 ** 12, "tokens": 1000}
+        v = bench.value_of("decode_128", work, ms, got_world)
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+        out_q.put((rank, got_world, got_rank, ms, e2e, v))
+    except Exception as e:  # report instead of hanging the parent
+        out_q.put((rank, "error", repr(e)))
+
+
+def test_two_replicas_take_the_slowest_rank():
+    """Each replica times its own steps; the job's step time is the max over
+    ranks and the value counts the work of every rank (weak scaling)."""
+    world, port = 2, _free_port()
+    ms_by_rank = [0.40, 0.55]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, ms_by_rank, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for r in res:
+        assert r[1] != "error", r
+        rank, got_world, got_rank, ms, e2e, v = r
+        assert got_world == 2 and got_rank == rank
+        assert ms == pytest.approx(0.55)
+        assert e2e == pytest.approx(1.10)
+        # 2 ranks x 1 GB each in 0.55 ms
+        assert v == pytest.approx(2 * 1e9 / 0.55e-3 / 1e9)
+
+
+def test_single_process_max_is_identity():
+    assert not torch.distributed.is_initialized()
+    assert bench.max_over_ranks(0.123, "cpu") == 0.123
+
+
+def test_algorithmic_counts_tiny_workload():
+    """Bytes and FLOPs of the tiny fp32 mix, counted by hand from its lengths:
+    (q, kv) = (1,37), (1,100), (50,50), (17,80); Hq 4, Hkv 1, D 64, page 16."""
+    prob = I.make_workload("tiny_mixed_f32", device="cpu")
+    w = bench.algorithmic(prob)
+    e, hq, hkv, d = 4, 4, 1, 64
+    q = np.array([1, 1, 50, 17])
+    k = np.array([37, 100, 50, 80])
+    assert list(prob.q_lens) == list(q) and list(prob.kv_lens) == list(k)
+    t = int(q.sum())
+    pages = int(((k + 15) // 16).sum())
+    want_bytes = (k.sum() * hkv * d * 2 * e + t * hkv * d * 2 * e + 2 * t * hq * d * e + 4 * t * hq
+                  + 4 * pages)
+    assert w["bytes"] == want_bytes
+    # causal visible pairs: decode rows see everything; prefill rows see c + i + 1 keys
+    pairs = 37 + 100 + sum(i + 1 for i in range(50)) + sum(63 + i + 1 for i in range(17))
+    assert w["flops"] == 4 * d * hq * pairs
+    assert w["tokens"] == t
+    assert w["prefill_flops"] == 4 * d * hq * (pairs - 37 - 100)
+
+
+def test_roofline_uses_the_dominant_kernel():
+    work = {"bytes": 3 * 10 ** 9, "flops": 4 * 10 ** 12, "tokens": 10, "decode_kernel_bytes": 2 * 10 ** 9,
+            "prefill_flops": 10 ** 12}
+    pk = {"hbm": 8000.0, "tc": 2000.0, "tc_sustained": 1500.0, "source": "test"}
+    # decode dominates: 2 launches of 0.25 ms each move 2 GB per launch
+    r = bench.roofline("decode_128", work, {"decode": (2, 0.5), "combine": (2, 0.05)}, pk)
+    assert r["kernel"] == "decode" and r["bound"] == "hbm"
+    assert r["achieved"] == pytest.approx(2e9 / 0.25e-3 / 1e9)
+    assert r["frac"] == pytest.approx(r["achieved"] / 8000.0)
+    # prefill dominates: 1 launch of 1 ms does 1 TFLOP
+    r = bench.roofline("mixed_96d_4c", work, {"decode": (1, 0.2), "prefill": (1, 1.0)}, pk)
+    assert r["kernel"] == "prefill" and r["bound"] == "tensor"
+    assert r["achieved"] == pytest.approx(1000.0)
+    assert r["kernel_share"]["prefill"] == pytest.approx(1.0 / 1.2, abs=1e-4)
