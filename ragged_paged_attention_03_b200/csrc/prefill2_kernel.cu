@@ -335,7 +335,16 @@ __global__ void __launch_bounds__(384, 1)
             ptx::tma_load_3d_elect(sQ + t * S::kQBytes + hh * BM * 128, &tm_q, &bars->q_full, hh * 64, w.h,
                                    w.tile.q_start + w.r0 + t * BM);
         }
+        // page of this lane's segment of context block j (-1: no segment);
+        // block j+1's entries are read while block j is issued
+        auto page_of = [&](int j) -> int {
+          const int sp = j * BN + lane * br;
+          return (j < w.n_ctx && lane < nseg && sp < w.c) ? pt_row[sp / pb.p] : -1;
+        };
+        int page_next = page_of(0);
         for (int j = 0; j < w.nb; ++j, ++g) {
+          const int page = page_next;
+          if (j + 1 < w.nb) page_next = page_of(j + 1);
           const int sk = g % NSK, sv = g % NSV;
           const uint32_t phk = (uint32_t)((g / NSK) & 1), phv = (uint32_t)((g / NSV) & 1);
           uint8_t *dk = sK + sk * S::kKVBytes;
@@ -343,18 +352,13 @@ __global__ void __launch_bounds__(384, 1)
           const bool ctx = j < w.n_ctx;
           const int pos0 = ctx ? j * BN : (j - w.n_ctx) * BN;
           const int valid = min(BN, (ctx ? w.c : w.tile.q_len) - pos0);
-          int page = -1;
           bool seg_loaded = false, seg_bad = false;
-          if (ctx && lane < nseg) {
-            const int sp = pos0 + lane * br;
-            if (sp < w.c) {
-              page = pt_row[sp / pb.p];
-              if (page < 0 || page >= pb.num_pages) {
-                seg_bad = true;
-                atomicOr(pb.err, RPA_DEV_BAD_PAGE);
-              } else {
-                seg_loaded = true;
-              }
+          if (ctx && lane < nseg && pos0 + lane * br < w.c) {
+            if (page < 0 || page >= pb.num_pages) {
+              seg_bad = true;
+              atomicOr(pb.err, RPA_DEV_BAD_PAGE);
+            } else {
+              seg_loaded = true;
             }
           }
           const unsigned loaded_mask = __ballot_sync(0xffffffffu, seg_loaded);
