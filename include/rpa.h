@@ -182,10 +182,16 @@ enum {
                                       RPA_OPT_CONCURRENT_MIXED is on (0 =
                                       chosen from the batch's estimated FLOPs
                                       and bytes) */
-  RPA_OPT_CONCURRENT_MIXED = 4     /* 1: run the prefill and decode work of a
+  RPA_OPT_CONCURRENT_MIXED = 4,    /* 1: run the prefill and decode work of a
                                       mixed batch concurrently on two streams
                                       (default 0: one after the other, faster
                                       on the measured mixes) */
+  RPA_OPT_PREFILL_LOADERS = 5      /* TMA producer warps of the head_dim <= 128
+                                      prefill kernel: 1 (K and V share one), 2
+                                      (one each; the cache update gets one warp
+                                      instead of two), 0 = chosen per batch:
+                                      2 when the prefill rows' cached context
+                                      outnumbers their new tokens (default 0) */
 };
 RPA_API int64_t rpa_set_option(int32_t option, int64_t value);
 

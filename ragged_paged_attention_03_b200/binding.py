@@ -28,6 +28,7 @@ RPA_OPT_FORCE_GENERIC = 1
 RPA_OPT_DISABLE_PREFILL_TC = 2
 RPA_OPT_PREFILL_SMS = 3
 RPA_OPT_CONCURRENT_MIXED = 4
+RPA_OPT_PREFILL_LOADERS = 5
 
 
 class rpa_dims(ctypes.Structure):

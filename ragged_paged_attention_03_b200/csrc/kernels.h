@@ -44,9 +44,10 @@ cudaError_t launch_prefill(const Problem &pb, const PrefillTile *tiles,
                            int n_tiles, cudaStream_t stream);
 
 // head_dim 64 / 128: two 128-row tiles per CTA (a 256-row work item);
-// persistent, at most max_ctas CTAs (<= 0: one per SM).
+// persistent, at most max_ctas CTAs (<= 0: one per SM).  split: K and V get
+// a producer warp each (for context-heavy batches) instead of sharing one.
 cudaError_t launch_prefill2(const Problem &pb, const PrefillTile *tiles,
-                            int n_tiles, int max_ctas, cudaStream_t stream);
+                            int n_tiles, int max_ctas, bool split, cudaStream_t stream);
 
 // Rows of a single prefill tile (query tokens per TMEM accumulator).
 constexpr int kPrefillTileRows = 128;

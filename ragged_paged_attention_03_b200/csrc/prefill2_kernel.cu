@@ -14,6 +14,10 @@
 //   warp 9                   TMEM owner and MMA issue
 //   warps 10-11              fused cache update: this CTA's share of the new
 //                            K/V rows copied into their page slots
+// A second build of the kernel (SPLIT) gives V a producer of its own in warp
+// 10, leaving warp 11 to the cache update: the planner picks it for batches
+// whose prefill work is mostly paged context (latency-bound gathers, few new
+// rows to write), the first one otherwise.
 // The producer and MMA warps run their loops with all 32 lanes and let one
 // elected lane issue each TMA copy, MMA, commit and arrive: a single-lane
 // branch would keep the operands in per-thread registers and cost many issue
@@ -60,7 +64,7 @@ struct Bars2 {
   uint64_t q_full, q_empty;
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
   uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];
-  uint64_t fix, drain;
+  uint64_t fix[2], drain;   // fix[1]: the V producer's, when V has its own warp
 };
 
 __device__ __forceinline__ bool wait_bar2(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
@@ -244,6 +248,315 @@ __device__ __forceinline__ void mma_loop(Bars2 *bars, volatile int *abort_flag, 
   __syncwarp();
 }
 
+// One producer warp for both operands: for every block, K as soon as its
+// stage is free, then V.  The Q tiles of each unit first.  Context blocks are
+// gathered one page segment per box through the page table (block j+1's
+// entries are read while block j is issued); a block with rows that hold no
+// valid key (past the context or the sequence, or on a page outside the
+// pool) goes through a private barrier: the copies land, the rows are zeroed,
+// then the block is published.
+template <int D>
+__device__ __forceinline__ void produce_kv(Bars2 *bars, volatile int *abort_flag, const Problem pb,
+                                           const PrefillTile *tiles, int n_units, uint8_t *sQ, uint8_t *sK,
+                                           uint8_t *sV, const CUtensorMap *tmq, const CUtensorMap *tmkc,
+                                           const CUtensorMap *tmvc, const CUtensorMap *tmkn, const CUtensorMap *tmvn) {
+  using S = P2Shape<D>;
+  constexpr int BM = S::BM, BN = S::BN, NSK = S::NSK, NSV = S::NSV;
+  const CUtensorMap &tm_q = *tmq, &tm_kc = *tmkc, &tm_vc = *tmvc, &tm_kn = *tmkn, &tm_vn = *tmvn;
+  const int lane = threadIdx.x & 31;
+  const int br = pb.p < BN ? pb.p : BN;
+  const int nseg = BN / br;
+  uint32_t fix_phase = 0;
+  int g = 0;            // K/V blocks started so far (all units)
+  int gk = 0, gv = 0;   // blocks whose K (V) copies were queued and published
+  bool fix_pending = false;
+  int uq = 0;           // units started
+  bool ok = true;
+  for (int r = 0, u = unit_of(0); ok && u < n_units; u = unit_of(++r), ++uq) {
+    const Unit w = make_unit<BM, BN>(tiles, u, pb);
+    const int32_t *pt_row = pb.page_table + (size_t)w.tile.seq * pb.max_pages;
+    // Q of both tiles, once the previous unit's QK MMAs are done with sQ
+    if (uq > 0 && !wait_all(&bars->q_empty, (uint32_t)((uq - 1) & 1), abort_flag, pb.err)) break;
+    ptx::mbar_arrive_expect_tx_elect(&bars->q_full, (w.rows_t[1] > 0 ? 2 : 1) * S::kQBytes);
+    for (int t = 0; t < 2; ++t) {
+      if (w.rows_t[t] == 0) continue;
+      for (int hh = 0; hh < S::kHalves; ++hh)
+        ptx::tma_load_3d_elect(sQ + t * S::kQBytes + hh * BM * 128, &tm_q, &bars->q_full, hh * 64, w.h,
+                               w.tile.q_start + w.r0 + t * BM);
+    }
+    // page of this lane's segment of context block j (-1: no segment);
+    // block j+1's entries are read while block j is issued
+    auto page_of = [&](int j) -> int {
+      const int sp = j * BN + lane * br;
+      return (j < w.n_ctx && lane < nseg && sp < w.c) ? pt_row[sp / pb.p] : -1;
+    };
+    int page_next = page_of(0);
+    for (int j = 0; j < w.nb; ++j, ++g) {
+      const int page = page_next;
+      if (j + 1 < w.nb) page_next = page_of(j + 1);
+      const int sk = g % NSK, sv = g % NSV;
+      const uint32_t phk = (uint32_t)((g / NSK) & 1), phv = (uint32_t)((g / NSV) & 1);
+      uint8_t *dk = sK + sk * S::kKVBytes;
+      uint8_t *dv = sV + sv * S::kKVBytes;
+      const bool ctx = j < w.n_ctx;
+      const int pos0 = ctx ? j * BN : (j - w.n_ctx) * BN;
+      const int valid = min(BN, (ctx ? w.c : w.tile.q_len) - pos0);
+      bool seg_loaded = false, seg_bad = false;
+      if (ctx && lane < nseg && pos0 + lane * br < w.c) {
+        if (page < 0 || page >= pb.num_pages) {
+          seg_bad = true;
+          atomicOr(pb.err, RPA_DEV_BAD_PAGE);
+        } else {
+          seg_loaded = true;
+        }
+      }
+      const unsigned loaded_mask = __ballot_sync(0xffffffffu, seg_loaded);
+      const bool fix = valid < BN || __any_sync(0xffffffffu, seg_bad);
+      const uint32_t seg_bytes = (uint32_t)(S::kHalves * br * 128);
+      const uint32_t blk_bytes = ctx ? (uint32_t)__popc(loaded_mask) * seg_bytes : (uint32_t)S::kKVBytes;
+      // the copies of one operand (K or V) of this block into dst
+      auto load = [&](uint8_t *dst, const CUtensorMap *tm_new, const CUtensorMap *tm_ctx, uint64_t *bar) {
+        if (!ctx) {
+          const int row = w.tile.q_start + pos0;
+          for (int hh = 0; hh < S::kHalves; ++hh)
+            ptx::tma_load_3d_elect(dst + hh * BN * 128, tm_new, bar, hh * 64, w.hk, row);
+        } else {
+          for (int sg = 0; sg < nseg; ++sg) {
+            const int pg = __shfl_sync(0xffffffffu, page, sg);
+            if (!((loaded_mask >> sg) & 1u)) continue;
+            const int sp = pos0 + sg * br;
+            const int row = pg * pb.p + (sp % pb.p);
+            for (int hh = 0; hh < S::kHalves; ++hh)
+              ptx::tma_load_3d_elect(dst + hh * BN * 128 + sg * br * 128, tm_ctx, bar, hh * 64, w.hk, row);
+          }
+        }
+      };
+      if (!fix) {
+        // K as soon as its stage is free, then V
+        if (g >= NSK && !wait_all(&bars->k_empty[sk], phk ^ 1u, abort_flag, pb.err)) {
+          ok = false;
+          break;
+        }
+        ptx::mbar_arrive_expect_tx_elect(&bars->k_full[sk], blk_bytes);
+        load(dk, &tm_kn, &tm_kc, &bars->k_full[sk]);
+        ++gk;
+        if (g >= NSV && !wait_all(&bars->v_empty[sv], phv ^ 1u, abort_flag, pb.err)) {
+          ok = false;
+          break;
+        }
+        ptx::mbar_arrive_expect_tx_elect(&bars->v_full[sv], blk_bytes);
+        load(dv, &tm_vn, &tm_vc, &bars->v_full[sv]);
+        ++gv;
+        continue;
+      }
+      // Partial block or bad pages: both operands through the private
+      // barrier, then zero the rows without a valid key and publish.
+      if ((g >= NSK && !wait_all(&bars->k_empty[sk], phk ^ 1u, abort_flag, pb.err)) ||
+          (g >= NSV && !wait_all(&bars->v_empty[sv], phv ^ 1u, abort_flag, pb.err))) {
+        ok = false;
+        break;
+      }
+      ptx::mbar_arrive_expect_tx_elect(&bars->fix[0], 2 * blk_bytes);
+      load(dk, &tm_kn, &tm_kc, &bars->fix[0]);
+      load(dv, &tm_vn, &tm_vc, &bars->fix[0]);
+      // the private barrier completes even when no copy was queued
+      const bool fok = wait_all(&bars->fix[0], fix_phase, abort_flag, pb.err);
+      fix_phase ^= 1u;
+      if (!fok) {
+        // copies may still be in flight: the drain below waits for them
+        fix_pending = true;
+        ok = false;
+        break;
+      }
+      for (int r = lane; r < BN; r += 32) {
+        const bool bad_row = r >= valid || (ctx && !((loaded_mask >> (r / br)) & 1u));
+        if (!bad_row) continue;
+        for (int hh = 0; hh < S::kHalves; ++hh) {
+          uint4 *pk = reinterpret_cast<uint4 *>(dk + hh * BN * 128 + r * 128);
+          uint4 *pv = reinterpret_cast<uint4 *>(dv + hh * BN * 128 + r * 128);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            pk[q] = make_uint4(0, 0, 0, 0);
+            pv[q] = make_uint4(0, 0, 0, 0);
+          }
+        }
+      }
+      ptx::fence_proxy_async_smem();
+      __syncwarp();
+      ptx::mbar_arrive_elect(&bars->k_full[sk]);
+      ptx::mbar_arrive_elect(&bars->v_full[sv]);
+      ++gk;
+      ++gv;
+    }
+  }
+  // every copy this warp queued must land before the CTA ends
+  if (lane == 0) {
+    if (uq > 0) ptx::mbar_wait(&bars->q_full, (uint32_t)((uq - 1) & 1));
+    for (int k = gk - NSK < 0 ? 0 : gk - NSK; k < gk; ++k)
+      ptx::mbar_wait(&bars->k_full[k % NSK], (uint32_t)((k / NSK) & 1));
+    for (int k = gv - NSV < 0 ? 0 : gv - NSV; k < gv; ++k)
+      ptx::mbar_wait(&bars->v_full[k % NSV], (uint32_t)((k / NSV) & 1));
+    if (fix_pending) ptx::mbar_wait(&bars->fix[0], fix_phase ^ 1u);
+  }
+  __syncwarp();
+}
+
+// One producer warp per operand (IS_V: V, else Q and K): each ring is filled
+// as soon as its own stages are released, so K runs a full ring ahead of
+// the QKs whatever the V ring waits for.  Used for batches whose prefill work
+// is mostly paged context, where the gathers are latency-bound.  Same block
+// handling as produce_kv, with a private barrier per operand.
+template <int D, bool IS_V>
+__device__ __forceinline__ void produce(Bars2 *bars, volatile int *abort_flag, const Problem pb,
+                                        const PrefillTile *tiles, int n_units, uint8_t *sQ, uint8_t *sOp,
+                                        const CUtensorMap *tm_q, const CUtensorMap *tm_new,
+                                        const CUtensorMap *tm_ctx) {
+  using S = P2Shape<D>;
+  constexpr int BM = S::BM, BN = S::BN, NS = IS_V ? S::NSV : S::NSK;
+  uint64_t *full = IS_V ? bars->v_full : bars->k_full;
+  uint64_t *empty = IS_V ? bars->v_empty : bars->k_empty;
+  uint64_t *fixb = &bars->fix[IS_V ? 1 : 0];
+  const int lane = threadIdx.x & 31;
+  const int br = pb.p < BN ? pb.p : BN;
+  const int nseg = BN / br;
+  uint32_t fix_phase = 0;
+  int g = 0;            // blocks started so far (all units)
+  int gp = 0;           // blocks whose copies were queued and published
+  bool fix_pending = false;
+  int uq = 0;           // units started
+  bool ok = true;
+  for (int r = 0, u = unit_of(0); ok && u < n_units; u = unit_of(++r), ++uq) {
+    const Unit w = make_unit<BM, BN>(tiles, u, pb);
+    const int32_t *pt_row = pb.page_table + (size_t)w.tile.seq * pb.max_pages;
+    if (!IS_V) {
+      // Q of both tiles, once the previous unit's QK MMAs are done with sQ
+      if (uq > 0 && !wait_all(&bars->q_empty, (uint32_t)((uq - 1) & 1), abort_flag, pb.err)) break;
+      ptx::mbar_arrive_expect_tx_elect(&bars->q_full, (w.rows_t[1] > 0 ? 2 : 1) * S::kQBytes);
+      for (int t = 0; t < 2; ++t) {
+        if (w.rows_t[t] == 0) continue;
+        for (int hh = 0; hh < S::kHalves; ++hh)
+          ptx::tma_load_3d_elect(sQ + t * S::kQBytes + hh * BM * 128, tm_q, &bars->q_full, hh * 64, w.h,
+                                 w.tile.q_start + w.r0 + t * BM);
+      }
+    }
+    // page of this lane's segment of context block j (-1: no such segment)
+    auto page_of = [&](int j) -> int {
+      const int sp = j * BN + lane * br;
+      return (j < w.n_ctx && lane < nseg && sp < w.c) ? pt_row[sp / pb.p] : -1;
+    };
+    int page_next = page_of(0);
+    for (int j = 0; j < w.nb; ++j, ++g) {
+      const int page = page_next;
+      if (j + 1 < w.nb) page_next = page_of(j + 1);
+      const int s = g % NS;
+      const uint32_t ph = (uint32_t)((g / NS) & 1);
+      uint8_t *dst = sOp + s * S::kKVBytes;
+      const bool ctx = j < w.n_ctx;
+      const int pos0 = ctx ? j * BN : (j - w.n_ctx) * BN;
+      const int valid = min(BN, (ctx ? w.c : w.tile.q_len) - pos0);
+      bool seg_loaded = false, seg_bad = false;
+      if (ctx && lane < nseg && pos0 + lane * br < w.c) {
+        if (page < 0 || page >= pb.num_pages) {
+          seg_bad = true;
+          if (!IS_V) atomicOr(pb.err, RPA_DEV_BAD_PAGE);
+        } else {
+          seg_loaded = true;
+        }
+      }
+      const unsigned loaded_mask = __ballot_sync(0xffffffffu, seg_loaded);
+      const bool fix = valid < BN || __any_sync(0xffffffffu, seg_bad);
+      const uint32_t seg_bytes = (uint32_t)(S::kHalves * br * 128);
+      const uint32_t blk_bytes = ctx ? (uint32_t)__popc(loaded_mask) * seg_bytes : (uint32_t)S::kKVBytes;
+      if (g >= NS && !wait_all(&empty[s], ph ^ 1u, abort_flag, pb.err)) {
+        ok = false;
+        break;
+      }
+      uint64_t *bar = fix ? fixb : &full[s];
+      ptx::mbar_arrive_expect_tx_elect(bar, blk_bytes);
+      if (!ctx) {
+        const int row = w.tile.q_start + pos0;
+        for (int hh = 0; hh < S::kHalves; ++hh)
+          ptx::tma_load_3d_elect(dst + hh * BN * 128, tm_new, bar, hh * 64, w.hk, row);
+      } else {
+        for (int sg = 0; sg < nseg; ++sg) {
+          const int pg = __shfl_sync(0xffffffffu, page, sg);
+          if (!((loaded_mask >> sg) & 1u)) continue;
+          const int sp = pos0 + sg * br;
+          const int row = pg * pb.p + (sp % pb.p);
+          for (int hh = 0; hh < S::kHalves; ++hh)
+            ptx::tma_load_3d_elect(dst + hh * BN * 128 + sg * br * 128, tm_ctx, bar, hh * 64, w.hk, row);
+        }
+      }
+      if (fix) {
+        // the private barrier completes even when no copy was queued
+        const bool fok = wait_all(fixb, fix_phase, abort_flag, pb.err);
+        fix_phase ^= 1u;
+        if (!fok) {
+          fix_pending = true;   // copies may still be in flight: drained below
+          ok = false;
+          break;
+        }
+        for (int rr = lane; rr < BN; rr += 32) {
+          const bool bad_row = rr >= valid || (ctx && !((loaded_mask >> (rr / br)) & 1u));
+          if (!bad_row) continue;
+          for (int hh = 0; hh < S::kHalves; ++hh) {
+            uint4 *pz = reinterpret_cast<uint4 *>(dst + hh * BN * 128 + rr * 128);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) pz[q] = make_uint4(0, 0, 0, 0);
+          }
+        }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        ptx::mbar_arrive_elect(&full[s]);
+      }
+      ++gp;
+    }
+  }
+  // every copy this warp queued must land before the CTA ends
+  if (lane == 0) {
+    if (!IS_V && uq > 0) ptx::mbar_wait(&bars->q_full, (uint32_t)((uq - 1) & 1));
+    for (int k = gp - NS < 0 ? 0 : gp - NS; k < gp; ++k) ptx::mbar_wait(&full[k % NS], (uint32_t)((k / NS) & 1));
+    if (fix_pending) ptx::mbar_wait(fixb, fix_phase ^ 1u);
+  }
+  __syncwarp();
+}
+
+// The fused cache update: threads [0, n) of the cache-writer warps copy this
+// CTA's share of the new K/V rows (one of the G query heads of each KV head
+// takes each row of an item) from k_new / v_new into their page slots.
+template <int D>
+__device__ __forceinline__ void cache_update(const Problem pb, const PrefillTile *tiles, int n_units, int wt,
+                                             int n) {
+  using S = P2Shape<D>;
+  constexpr int BM = S::BM, BN = S::BN;
+  const int G = pb.hq / pb.hkv;
+  const int chunks = D / 8;
+  const __nv_bfloat16 *kn = reinterpret_cast<const __nv_bfloat16 *>(pb.k_new);
+  const __nv_bfloat16 *vn = reinterpret_cast<const __nv_bfloat16 *>(pb.v_new);
+  __nv_bfloat16 *kc = reinterpret_cast<__nv_bfloat16 *>(pb.k_cache);
+  __nv_bfloat16 *vc = reinterpret_cast<__nv_bfloat16 *>(pb.v_cache);
+  for (int r = 0, u = unit_of(0); u < n_units; u = unit_of(++r)) {
+    const Unit w = make_unit<BM, BN>(tiles, u, pb);
+    const int32_t *pt_row = pb.page_table + (size_t)w.tile.seq * pb.max_pages;
+    const int gidx = w.h % G;
+    const int ra = (gidx * w.tile.rows) / G, rb = ((gidx + 1) * w.tile.rows) / G;
+    for (int idx = wt; idx < (rb - ra) * chunks; idx += n) {
+      const int i = w.r0 + ra + idx / chunks;   // new-token index
+      const int ch = idx % chunks;
+      const int pos = w.c + i;
+      const int pg = pt_row[pos / pb.p];
+      if (pg < 0 || pg >= pb.num_pages) {
+        if (ch == 0) atomicOr(pb.err, RPA_DEV_BAD_PAGE);
+        continue;
+      }
+      const size_t src = ((size_t)(w.tile.q_start + i) * pb.hkv + w.hk) * D + ch * 8;
+      const size_t dst = (((size_t)pg * pb.p + pos % pb.p) * pb.hkv + w.hk) * D + ch * 8;
+      *reinterpret_cast<uint4 *>(kc + dst) = *reinterpret_cast<const uint4 *>(kn + src);
+      *reinterpret_cast<uint4 *>(vc + dst) = *reinterpret_cast<const uint4 *>(vn + src);
+    }
+  }
+}
+
 // Persistent: each CTA walks its units in the order of unit_of() over the
 // list of (item, query head) units; items are sorted heaviest first on the
 // host and the heads of one item are consecutive (their K/V blocks are
@@ -251,7 +564,7 @@ __device__ __forceinline__ void mma_loop(Bars2 *bars, volatile int *abort_flag, 
 // Every barrier parity runs on counters that span units, so the producer
 // loads the next unit's Q and K/V while the current one finishes and the MMA
 // warp starts the next unit while the softmax warps are still storing O.
-template <int D>
+template <int D, bool SPLIT>
 __global__ void __launch_bounds__(384, 1)
     prefill2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
                     const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_kn,
@@ -271,7 +584,6 @@ __global__ void __launch_bounds__(384, 1)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int G = pb.hq / pb.hkv;
 
   if (tid == 0) {
     ptx::mbar_init(&bars->q_full, 1);
@@ -290,7 +602,8 @@ __global__ void __launch_bounds__(384, 1)
       ptx::mbar_init(&bars->pv_done[i], 1);
       ptx::mbar_init(&bars->o_free[i], 128);
     }
-    ptx::mbar_init(&bars->fix, 1);
+    ptx::mbar_init(&bars->fix[0], 1);
+    ptx::mbar_init(&bars->fix[1], 1);
     ptx::mbar_init(&bars->drain, 1);
     *abort_flag = 0;
     ptx::fence_barrier_init();
@@ -314,174 +627,19 @@ __global__ void __launch_bounds__(384, 1)
   if (warp >= 8) {
     setmaxnreg_dec96();
     if (warp == 8) {
-      // ---------------------------------------------------------- producer
-      const int br = pb.p < BN ? pb.p : BN;
-      const int nseg = BN / br;
-      uint32_t fix_phase = 0;
-      int g = 0;            // K/V blocks started so far (all units)
-      int gk = 0, gv = 0;   // blocks whose K (V) copies were queued and published
-      bool fix_pending = false;
-      int uq = 0;           // units started
-      bool ok = true;
-      for (int r = 0, u = unit_of(0); ok && u < n_units; u = unit_of(++r), ++uq) {
-        const Unit w = make_unit<BM, BN>(tiles, u, pb);
-        const int32_t *pt_row = pb.page_table + (size_t)w.tile.seq * pb.max_pages;
-        // Q of both tiles, once the previous unit's QK MMAs are done with sQ
-        if (uq > 0 && !wait_all(&bars->q_empty, (uint32_t)((uq - 1) & 1), abort_flag, pb.err)) break;
-        ptx::mbar_arrive_expect_tx_elect(&bars->q_full, (w.rows_t[1] > 0 ? 2 : 1) * S::kQBytes);
-        for (int t = 0; t < 2; ++t) {
-          if (w.rows_t[t] == 0) continue;
-          for (int hh = 0; hh < S::kHalves; ++hh)
-            ptx::tma_load_3d_elect(sQ + t * S::kQBytes + hh * BM * 128, &tm_q, &bars->q_full, hh * 64, w.h,
-                                   w.tile.q_start + w.r0 + t * BM);
-        }
-        // page of this lane's segment of context block j (-1: no segment);
-        // block j+1's entries are read while block j is issued
-        auto page_of = [&](int j) -> int {
-          const int sp = j * BN + lane * br;
-          return (j < w.n_ctx && lane < nseg && sp < w.c) ? pt_row[sp / pb.p] : -1;
-        };
-        int page_next = page_of(0);
-        for (int j = 0; j < w.nb; ++j, ++g) {
-          const int page = page_next;
-          if (j + 1 < w.nb) page_next = page_of(j + 1);
-          const int sk = g % NSK, sv = g % NSV;
-          const uint32_t phk = (uint32_t)((g / NSK) & 1), phv = (uint32_t)((g / NSV) & 1);
-          uint8_t *dk = sK + sk * S::kKVBytes;
-          uint8_t *dv = sV + sv * S::kKVBytes;
-          const bool ctx = j < w.n_ctx;
-          const int pos0 = ctx ? j * BN : (j - w.n_ctx) * BN;
-          const int valid = min(BN, (ctx ? w.c : w.tile.q_len) - pos0);
-          bool seg_loaded = false, seg_bad = false;
-          if (ctx && lane < nseg && pos0 + lane * br < w.c) {
-            if (page < 0 || page >= pb.num_pages) {
-              seg_bad = true;
-              atomicOr(pb.err, RPA_DEV_BAD_PAGE);
-            } else {
-              seg_loaded = true;
-            }
-          }
-          const unsigned loaded_mask = __ballot_sync(0xffffffffu, seg_loaded);
-          const bool fix = valid < BN || __any_sync(0xffffffffu, seg_bad);
-          const uint32_t seg_bytes = (uint32_t)(S::kHalves * br * 128);
-          const uint32_t blk_bytes = ctx ? (uint32_t)__popc(loaded_mask) * seg_bytes : (uint32_t)S::kKVBytes;
-          // the copies of one operand (K or V) of this block into dst
-          auto load = [&](uint8_t *dst, const CUtensorMap *tm_new, const CUtensorMap *tm_ctx, uint64_t *bar) {
-            if (!ctx) {
-              const int row = w.tile.q_start + pos0;
-              for (int hh = 0; hh < S::kHalves; ++hh)
-                ptx::tma_load_3d_elect(dst + hh * BN * 128, tm_new, bar, hh * 64, w.hk, row);
-            } else {
-              for (int sg = 0; sg < nseg; ++sg) {
-                const int pg = __shfl_sync(0xffffffffu, page, sg);
-                if (!((loaded_mask >> sg) & 1u)) continue;
-                const int sp = pos0 + sg * br;
-                const int row = pg * pb.p + (sp % pb.p);
-                for (int hh = 0; hh < S::kHalves; ++hh)
-                  ptx::tma_load_3d_elect(dst + hh * BN * 128 + sg * br * 128, tm_ctx, bar, hh * 64, w.hk, row);
-              }
-            }
-          };
-          if (!fix) {
-            // K as soon as its stage is free, then V
-            if (g >= NSK && !wait_all(&bars->k_empty[sk], phk ^ 1u, abort_flag, pb.err)) {
-              ok = false;
-              break;
-            }
-            ptx::mbar_arrive_expect_tx_elect(&bars->k_full[sk], blk_bytes);
-            load(dk, &tm_kn, &tm_kc, &bars->k_full[sk]);
-            ++gk;
-            if (g >= NSV && !wait_all(&bars->v_empty[sv], phv ^ 1u, abort_flag, pb.err)) {
-              ok = false;
-              break;
-            }
-            ptx::mbar_arrive_expect_tx_elect(&bars->v_full[sv], blk_bytes);
-            load(dv, &tm_vn, &tm_vc, &bars->v_full[sv]);
-            ++gv;
-            continue;
-          }
-          // Partial block or bad pages: both operands through the private
-          // barrier, then zero the rows without a valid key and publish.
-          if ((g >= NSK && !wait_all(&bars->k_empty[sk], phk ^ 1u, abort_flag, pb.err)) ||
-              (g >= NSV && !wait_all(&bars->v_empty[sv], phv ^ 1u, abort_flag, pb.err))) {
-            ok = false;
-            break;
-          }
-          ptx::mbar_arrive_expect_tx_elect(&bars->fix, 2 * blk_bytes);
-          load(dk, &tm_kn, &tm_kc, &bars->fix);
-          load(dv, &tm_vn, &tm_vc, &bars->fix);
-          // the private barrier completes even when no copy was queued
-          const bool fok = wait_all(&bars->fix, fix_phase, abort_flag, pb.err);
-          fix_phase ^= 1u;
-          if (!fok) {
-            // copies may still be in flight: the drain below waits for them
-            fix_pending = true;
-            ok = false;
-            break;
-          }
-          for (int r = lane; r < BN; r += 32) {
-            const bool bad_row = r >= valid || (ctx && !((loaded_mask >> (r / br)) & 1u));
-            if (!bad_row) continue;
-            for (int hh = 0; hh < S::kHalves; ++hh) {
-              uint4 *pk = reinterpret_cast<uint4 *>(dk + hh * BN * 128 + r * 128);
-              uint4 *pv = reinterpret_cast<uint4 *>(dv + hh * BN * 128 + r * 128);
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                pk[q] = make_uint4(0, 0, 0, 0);
-                pv[q] = make_uint4(0, 0, 0, 0);
-              }
-            }
-          }
-          ptx::fence_proxy_async_smem();
-          __syncwarp();
-          ptx::mbar_arrive_elect(&bars->k_full[sk]);
-          ptx::mbar_arrive_elect(&bars->v_full[sv]);
-          ++gk;
-          ++gv;
-        }
-      }
-      // every copy this warp queued must land before the CTA ends
-      if (lane == 0) {
-        if (uq > 0) ptx::mbar_wait(&bars->q_full, (uint32_t)((uq - 1) & 1));
-        for (int k = gk - NSK < 0 ? 0 : gk - NSK; k < gk; ++k)
-          ptx::mbar_wait(&bars->k_full[k % NSK], (uint32_t)((k / NSK) & 1));
-        for (int k = gv - NSV < 0 ? 0 : gv - NSV; k < gv; ++k)
-          ptx::mbar_wait(&bars->v_full[k % NSV], (uint32_t)((k / NSV) & 1));
-        if (fix_pending) ptx::mbar_wait(&bars->fix, fix_phase ^ 1u);
-      }
-      __syncwarp();
+      if (SPLIT)
+        produce<D, false>(bars, abort_flag, pb, tiles, n_units, sQ, sK, &tm_q, &tm_kn, &tm_kc);
+      else
+        produce_kv<D>(bars, abort_flag, pb, tiles, n_units, sQ, sK, sV, &tm_q, &tm_kc, &tm_vc, &tm_kn, &tm_vn);
     } else if (warp == 9) {
       // --------------------------------------------------------------- MMA
       mma_loop<D>(bars, abort_flag, pb, tiles, n_units, tmem, ptx::smem_u32(sQ), ptx::smem_u32(sK),
                   ptx::smem_u32(sV));
+    } else if (SPLIT && warp == 10) {
+      produce<D, true>(bars, abort_flag, pb, tiles, n_units, sQ, sV, &tm_q, &tm_vn, &tm_vc);
     } else {
-      // ------------------------------------------ fused cache update (64 thr)
-      const int chunks = D / 8;
-      const int wt = tid - 320;
-      const __nv_bfloat16 *kn = reinterpret_cast<const __nv_bfloat16 *>(pb.k_new);
-      const __nv_bfloat16 *vn = reinterpret_cast<const __nv_bfloat16 *>(pb.v_new);
-      __nv_bfloat16 *kc = reinterpret_cast<__nv_bfloat16 *>(pb.k_cache);
-      __nv_bfloat16 *vc = reinterpret_cast<__nv_bfloat16 *>(pb.v_cache);
-      for (int r = 0, u = unit_of(0); u < n_units; u = unit_of(++r)) {
-        const Unit w = make_unit<BM, BN>(tiles, u, pb);
-        const int32_t *pt_row = pb.page_table + (size_t)w.tile.seq * pb.max_pages;
-        const int gidx = w.h % G;
-        const int ra = (gidx * w.tile.rows) / G, rb = ((gidx + 1) * w.tile.rows) / G;
-        for (int idx = wt; idx < (rb - ra) * chunks; idx += 64) {
-          const int i = w.r0 + ra + idx / chunks;   // new-token index
-          const int ch = idx % chunks;
-          const int pos = w.c + i;
-          const int pg = pt_row[pos / pb.p];
-          if (pg < 0 || pg >= pb.num_pages) {
-            if (ch == 0) atomicOr(pb.err, RPA_DEV_BAD_PAGE);
-            continue;
-          }
-          const size_t src = ((size_t)(w.tile.q_start + i) * pb.hkv + w.hk) * D + ch * 8;
-          const size_t dst = (((size_t)pg * pb.p + pos % pb.p) * pb.hkv + w.hk) * D + ch * 8;
-          *reinterpret_cast<uint4 *>(kc + dst) = *reinterpret_cast<const uint4 *>(kn + src);
-          *reinterpret_cast<uint4 *>(vc + dst) = *reinterpret_cast<const uint4 *>(vn + src);
-        }
-      }
+      // fused cache update: warps 10-11, or warp 11 when warp 10 loads V
+      cache_update<D>(pb, tiles, n_units, SPLIT ? lane : tid - 320, SPLIT ? 32 : 64);
     }
   } else {
     // ----------------------------------------------------------- softmax
@@ -629,7 +787,8 @@ __global__ void __launch_bounds__(384, 1)
 }
 
 template <int D>
-cudaError_t launch_t(const Problem &pb, const PrefillTile *tiles, int n_tiles, int max_ctas, cudaStream_t stream) {
+cudaError_t launch_t(const Problem &pb, const PrefillTile *tiles, int n_tiles, int max_ctas, bool split,
+                     cudaStream_t stream) {
   using S = P2Shape<D>;
   CUtensorMap tq, tkc, tvc, tkn, tvn;
   const uint64_t qdims[3] = {(uint64_t)D, (uint64_t)pb.hq, (uint64_t)pb.total_q};
@@ -647,7 +806,7 @@ cudaError_t launch_t(const Problem &pb, const PrefillTile *tiles, int n_tiles, i
       !make_tmap_bf16_3d(&tkn, pb.k_new, ndims, nstr, nbox, true) ||
       !make_tmap_bf16_3d(&tvn, pb.v_new, ndims, nstr, nbox, true))
     return cudaErrorInvalidValue;
-  auto kern = prefill2_kernel<D>;
+  auto kern = split ? prefill2_kernel<D, true> : prefill2_kernel<D, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem);
   if (e != cudaSuccess) return e;
   const int n_units = n_tiles * pb.hq;
@@ -666,12 +825,12 @@ cudaError_t launch_t(const Problem &pb, const PrefillTile *tiles, int n_tiles, i
 
 }  // namespace
 
-cudaError_t launch_prefill2(const Problem &pb, const PrefillTile *tiles, int n_tiles, int max_ctas,
+cudaError_t launch_prefill2(const Problem &pb, const PrefillTile *tiles, int n_tiles, int max_ctas, bool split,
                             cudaStream_t stream) {
   if (n_tiles <= 0) return cudaSuccess;
   switch (pb.d) {
-    case 64: return launch_t<64>(pb, tiles, n_tiles, max_ctas, stream);
-    case 128: return launch_t<128>(pb, tiles, n_tiles, max_ctas, stream);
+    case 64: return launch_t<64>(pb, tiles, n_tiles, max_ctas, split, stream);
+    case 128: return launch_t<128>(pb, tiles, n_tiles, max_ctas, split, stream);
     default: return cudaErrorInvalidValue;
   }
 }

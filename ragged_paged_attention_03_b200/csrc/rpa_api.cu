@@ -29,6 +29,7 @@ std::atomic<int64_t> g_opt_force_generic{0};
 std::atomic<int64_t> g_opt_disable_prefill_tc{0};
 std::atomic<int64_t> g_opt_prefill_sms{0};
 std::atomic<int64_t> g_opt_concurrent_mixed{0};
+std::atomic<int64_t> g_opt_prefill_loaders{0};
 
 constexpr int kDefaultDecodeChunkBlocks = 128;
 // 256 blocks of 16 tokens touch at most 4096 / 8 + 1 pages, within the decode
@@ -104,6 +105,7 @@ struct HostPlan {
   int32_t num_decode = 0, num_prefill = 0, num_generic = 0, num_empty = 0;
   double decode_bytes = 0.0;     // K/V bytes the decode kernel streams
   double prefill_flops = 0.0;    // visible (q, k) pairs x 4 D Hq
+  int64_t prefill_ctx_tokens = 0, prefill_new_tokens = 0;
   PlanLayout layout{};
 };
 
@@ -168,6 +170,8 @@ void build_plan(const int32_t *cu, const int32_t *kv, int32_t n, const int32_t *
         {
           const double q = ql, c = (double)kvl - ql;
           hp.prefill_flops += 4.0 * d->head_dim * d->num_q_heads * q * (c + (q + 1) / 2.0);
+          hp.prefill_ctx_tokens += (int64_t)kvl - ql;
+          hp.prefill_new_tokens += ql;
         }
         const int32_t item_rows = prefill_item_rows(d->head_dim);
         for (int32_t r = 0; r < ql; r += item_rows) {
@@ -377,6 +381,7 @@ extern "C" RPA_API int64_t rpa_set_option(int32_t option, int64_t value) {
     case RPA_OPT_DISABLE_PREFILL_TC: return g_opt_disable_prefill_tc.exchange(value);
     case RPA_OPT_PREFILL_SMS: return g_opt_prefill_sms.exchange(value);
     case RPA_OPT_CONCURRENT_MIXED: return g_opt_concurrent_mixed.exchange(value);
+    case RPA_OPT_PREFILL_LOADERS: return g_opt_prefill_loaders.exchange(value);
     default: return -1;
   }
 }
@@ -486,7 +491,12 @@ extern "C" RPA_API int rpa_forward(const void *q, const void *k_new, const void 
     if (L.n_prefill_tiles > 0 && e == cudaSuccess)
       e = traced(RPA_KERNEL_PREFILL, pstream, [&] {
         const PrefillTile *tiles = (const PrefillTile *)(slot.dev + L.prefill_off);
-        return pb.d <= 128 ? launch_prefill2(pb, tiles, (int)L.n_prefill_tiles, prefill_ctas, pstream)
+        // context-heavy prefill (chunked rows after a long cache) gathers
+        // latency-bound paged blocks and writes few new rows: a producer warp
+        // per operand; fresh prefill keeps two warps for the cache update
+        const int64_t lo = g_opt_prefill_loaders.load();
+        const bool split = lo == 2 || (lo != 1 && hp.prefill_ctx_tokens > hp.prefill_new_tokens);
+        return pb.d <= 128 ? launch_prefill2(pb, tiles, (int)L.n_prefill_tiles, prefill_ctas, split, pstream)
                            : launch_prefill(pb, tiles, (int)L.n_prefill_tiles, pstream);
       });
     if (mixed && cudaEventRecord(slot.join, pstream) != cudaSuccess) e = cudaErrorUnknown;

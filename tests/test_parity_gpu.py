@@ -110,6 +110,38 @@ def test_decode_heavy_split_kv(oracle_mod, chunk):
         binding.rpa_set_option(binding.RPA_OPT_DECODE_CHUNK_BLOCKS, old)
 
 
+@pytest.mark.parametrize("loaders", [1, 2])
+@pytest.mark.parametrize("case", [4, 5, 6, 7, 8])
+def test_prefill_loader_builds(oracle_mod, loaders, case):
+    """Both builds of the head_dim <= 128 prefill kernel (K and V sharing one
+    producer warp, or one each), forced through RPA_OPT_PREFILL_LOADERS, on
+    fresh and chunked prefill mixes with ragged tails."""
+    from ragged_paged_attention_03_b200 import binding
+    old = binding.rpa_set_option(binding.RPA_OPT_PREFILL_LOADERS, loaders)
+    try:
+        ql, kv, hq, hkv, d, p, causal = SMALL[case]
+        prob = I.make_problem(ql, kv, num_q_heads=hq, num_kv_heads=hkv, head_dim=d, page_size=p,
+                              dtype=I.BF16, causal=causal, seed=300 + case, pool=1.5)
+        full_check(oracle_mod, prob)
+    finally:
+        binding.rpa_set_option(binding.RPA_OPT_PREFILL_LOADERS, old)
+
+
+@pytest.mark.parametrize("loaders", [1, 2])
+def test_chunked_prefill_long_context(oracle_mod, loaders):
+    """Chunked prefill after a long paged context (the batch shape that picks
+    one producer warp per operand), page size 8, with partial blocks at the
+    end of the context and of the new rows."""
+    from ragged_paged_attention_03_b200 import binding
+    old = binding.rpa_set_option(binding.RPA_OPT_PREFILL_LOADERS, loaders)
+    try:
+        prob = I.make_problem([300, 77, 1], [2100, 1000, 500], num_q_heads=16, num_kv_heads=4,
+                              head_dim=128, page_size=8, dtype=I.BF16, seed=41, pool=1.3)
+        full_check(oracle_mod, prob)
+    finally:
+        binding.rpa_set_option(binding.RPA_OPT_PREFILL_LOADERS, old)
+
+
 def test_bad_page_is_flagged_not_read(oracle_mod):
     """A page-table entry outside the pool is reported through the device
     error word; the kernels never dereference it."""
