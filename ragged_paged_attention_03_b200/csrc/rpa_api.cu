@@ -188,6 +188,11 @@ void build_plan(const int32_t *cu, const int32_t *kv, int32_t n, const int32_t *
       }
     }
   }
+  // Longest decode work items first: the kernel takes items in grid order,
+  // so the short ones fill the last wave instead of trailing it.
+  std::stable_sort(hp.decode.begin(), hp.decode.end(), [](const DecodeItem &a, const DecodeItem &b) {
+    return a.blk_end - a.blk_begin > b.blk_end - b.blk_begin;
+  });
   // Heaviest prefill tiles first: with a causal mask a tile's key range ends
   // at its last row, so later tiles of a sequence carry more work.
   std::stable_sort(hp.prefill.begin(), hp.prefill.end(),
