@@ -64,6 +64,7 @@ struct Bars2 {
   uint64_t q_full, q_empty;
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
   uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];
+  uint64_t p_half[2];   // P of keys 0..63 stored (PV's first four k-steps may start)
   uint64_t fix[2], drain;   // fix[1]: the V producer's, when V has its own warp
 };
 
@@ -156,13 +157,20 @@ __device__ __forceinline__ bool issue_pv(Bars2 *bars, volatile int *abort_flag, 
   using S = P2Shape<D>;
   constexpr uint32_t idesc = ptx::umma_idesc_bf16(128, D, true);
   const int s = gblk % S::NSV;
-  if (!wait_all(&bars->p_full[t], (uint32_t)(tblk & 1), abort_flag, err)) return false;
+  // P arrives in two halves: keys 0..63 feed the first four k-steps while
+  // the softmax warps still compute the rest
+  if (!wait_all(&bars->p_half[t], (uint32_t)(tblk & 1), abort_flag, err)) return false;
   if (wait_v && !wait_all(&bars->v_full[s], (uint32_t)((gblk / S::NSV) & 1), abort_flag, err)) return false;
   ptx::tc_fence_after();
   const uint64_t dv = dv0 + (uint64_t)((s * S::kKVBytes) >> 4);
 #pragma unroll
-  for (int kk = 0; kk < S::BN / 16; ++kk)
+  for (int kk = 0; kk < S::BN / 32; ++kk)
     ptx::umma_ts_elect(tO, tS + kk * 8, dv + (uint64_t)((kk * 16 * 128) >> 4), idesc, (!first || kk > 0) ? 1u : 0u);
+  if (!wait_all(&bars->p_full[t], (uint32_t)(tblk & 1), abort_flag, err)) return false;
+  ptx::tc_fence_after();
+#pragma unroll
+  for (int kk = S::BN / 32; kk < S::BN / 16; ++kk)
+    ptx::umma_ts_elect(tO, tS + kk * 8, dv + (uint64_t)((kk * 16 * 128) >> 4), idesc, 1u);
   return true;
 }
 
@@ -599,6 +607,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&bars->s_full[i], 1);
       ptx::mbar_init(&bars->p_full[i], 128);
+      ptx::mbar_init(&bars->p_half[i], 128);
       ptx::mbar_init(&bars->pv_done[i], 1);
       ptx::mbar_init(&bars->o_free[i], 128);
     }
@@ -724,18 +733,25 @@ __global__ void __launch_bounds__(384, 1)
         uint64_t sp2[4] = {0, 0, 0, 0};   // packed partial sums (+0.0f pairs)
         uint32_t pk[BN / 2];
 #pragma unroll
-        for (int i = 0; i < BN; i += 2) {
-          float a0, a1;
-          ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(x[i], x[i + 1]), scale2, negm2), a0, a1);
-          const uint64_t pp = ptx::f2_pack(ptx::ex2(a0), ptx::ex2(a1));
-          sp2[(i >> 1) & 3] = ptx::f2_add(sp2[(i >> 1) & 3], pp);
-          float p0, p1;
-          ptx::f2_unpack(pp, p0, p1);
-          pk[i >> 1] = ptx::pack_bf16(p0, p1);
-        }
+        for (int hf = 0; hf < 2; ++hf) {
 #pragma unroll
-        for (int cc = 0; cc < BN / 64; ++cc)
-          ptx::tmem_st32(tS + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[cc * 32]));
+          for (int i = hf * (BN / 2); i < (hf + 1) * (BN / 2); i += 2) {
+            float a0, a1;
+            ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(x[i], x[i + 1]), scale2, negm2), a0, a1);
+            const uint64_t pp = ptx::f2_pack(ptx::ex2(a0), ptx::ex2(a1));
+            sp2[(i >> 1) & 3] = ptx::f2_add(sp2[(i >> 1) & 3], pp);
+            float p0, p1;
+            ptx::f2_unpack(pp, p0, p1);
+            pk[i >> 1] = ptx::pack_bf16(p0, p1);
+          }
+          // P of keys [64 hf, 64 hf + 64) as bf16 into S's columns [32 hf, 32 hf + 32)
+          ptx::tmem_st32(tS + hf * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[hf * 32]));
+          if (hf == 0) {
+            ptx::tmem_st_wait();
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&bars->p_half[t]);
+          }
+        }
         float sp[8];
 #pragma unroll
         for (int k = 0; k < 4; ++k) ptx::f2_unpack(sp2[k], sp[2 * k], sp[2 * k + 1]);
