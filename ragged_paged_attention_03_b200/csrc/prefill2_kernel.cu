@@ -773,24 +773,24 @@ __global__ void __launch_bounds__(384, 1)
       const bool store = row < rows_mine;
       __nv_bfloat16 *out =
           reinterpret_cast<__nv_bfloat16 *>(pb.out) + ((size_t)(w.tile.q_start + rn) * pb.hq + w.h) * D;
+      // all of O_t into registers with one wait, then O_t is free for the
+      // next unit's first PV while the rows are stored
+      uint32_t ov[D];
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t r[32];
-        ptx::tmem_ld32(tO + cc * 32, r);
-        ptx::tmem_ld_wait();
-        if (store) {
-          uint32_t o2[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            o2[i] = ptx::pack_bf16(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
-          uint4 *dst = reinterpret_cast<uint4 *>(out + cc * 32);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(o2[4 * i], o2[4 * i + 1], o2[4 * i + 2], o2[4 * i + 3]);
-        }
-      }
-      // O has been read: the next unit's first PV may overwrite it
+      for (int cc = 0; cc < D / 32; ++cc) ptx::tmem_ld32(tO + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[cc * 32]));
+      ptx::tmem_ld_wait();
       ptx::tc_fence_before();
       ptx::mbar_arrive(&bars->o_free[t]);
+      if (store) {
+#pragma unroll
+        for (int cc = 0; cc < D / 8; ++cc) {
+          uint32_t o2[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            o2[i] = ptx::pack_bf16(__uint_as_float(ov[cc * 8 + 2 * i]) * inv, __uint_as_float(ov[cc * 8 + 2 * i + 1]) * inv);
+          reinterpret_cast<uint4 *>(out)[cc] = make_uint4(o2[0], o2[1], o2[2], o2[3]);
+        }
+      }
       ++ep;
       if (store && pb.lse != nullptr) pb.lse[(size_t)(w.tile.q_start + rn) * pb.hq + w.h] = (m + log2f(l)) * kLn2;
     }
