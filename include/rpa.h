@@ -173,7 +173,7 @@ RPA_API int rpa_plan(const int32_t *cu_q_lens, const int32_t *kv_lens,
 /* Planner knobs (process-wide).  Each returns the previous value. */
 enum {
   RPA_OPT_DECODE_CHUNK_BLOCKS = 0, /* 16-token blocks per decode work item
-                                      (default 128; <= 0 restores it) */
+                                      (default 192; <= 0 restores it) */
   RPA_OPT_FORCE_GENERIC = 1,       /* 1: run every sequence on the generic
                                       kernel (default 0) */
   RPA_OPT_DISABLE_PREFILL_TC = 2,  /* 1: prefill sequences use the generic

@@ -31,7 +31,7 @@ std::atomic<int64_t> g_opt_prefill_sms{0};
 std::atomic<int64_t> g_opt_concurrent_mixed{0};
 std::atomic<int64_t> g_opt_prefill_loaders{0};
 
-constexpr int kDefaultDecodeChunkBlocks = 128;
+constexpr int kDefaultDecodeChunkBlocks = 192;
 // 256 blocks of 16 tokens touch at most 4096 / 8 + 1 pages, within the decode
 // kernel's 1024-entry page list.
 constexpr int kMaxDecodeChunkBlocks = 256;
