@@ -102,6 +102,8 @@ typedef struct {
  *            technique 3).  NULL: the library classifies each sequence
  *            itself and sequence order does not matter.  It only chooses
  *            kernels; results never depend on it.
+ * scale: the factor on q.k (1/sqrt(D) for standard attention); it must be
+ *            positive and finite, otherwise RPA_ERR_INVALID_ARG.
  *
  * Semantics (exact attention; talk summary 00:06:36 for the order):
  *   1. for every s and i < q_len[s], K/V of new token cu_q_lens[s] + i are

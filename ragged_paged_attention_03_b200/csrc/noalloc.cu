@@ -66,6 +66,7 @@ extern "C" RPA_API int rpa_decode_noalloc(const void *q, const void *k_new, cons
   cudaStream_t stream = (cudaStream_t)stream_ptr;
   // ---- validation (host only)
   if (dims == nullptr || num_seqs < 0) return RPA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return RPA_ERR_INVALID_ARG;
   if (dims->dtype != RPA_BF16) return RPA_ERR_UNSUPPORTED;
   if (dims->num_q_heads <= 0 || dims->num_kv_heads <= 0 || dims->num_pages <= 0 ||
       dims->max_pages_per_seq <= 0)

@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(192, 1)
     // ---------------------------------------------------------------- MMA
     // All 32 lanes run the loop; one elected lane issues each MMA / commit.
     {
-      const uint32_t tS[2] = {tmem + S::kColS0, tmem + S::kColS1};
+      const uint32_t tS0 = tmem + S::kColS0, tS1 = tmem + S::kColS1;
       const uint32_t tO = tmem + S::kColO;
       constexpr uint32_t idesc_qk = ptx::umma_idesc_bf16(128, BN, false);
       constexpr uint32_t idesc_pv = ptx::umma_idesc_bf16(128, D, true);
@@ -277,18 +277,17 @@ __global__ void __launch_bounds__(192, 1)
         const uint64_t dv = dv0 + (uint64_t)((s * S::kKVBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          ptx::umma_ts_elect(tO, tS[b] + kk * 8, dv + (uint64_t)((kk * 16 * 128) >> 4), idesc_pv,
+          ptx::umma_ts_elect(tO, (b ? tS1 : tS0) + kk * 8, dv + (uint64_t)((kk * 16 * 128) >> 4), idesc_pv,
                              (i > 0 || kk > 0) ? 1u : 0u);
         ptx::umma_commit_elect(&bars->pv_done[b]);
         ptx::umma_commit_elect(&bars->v_empty[s]);
         return true;
       };
+      // QK(j) writes the S buffer that PV(j-2) reads P from; it is issued
+      // after PV(j-2) without waiting for it to finish, because tcgen05.mma
+      // operations issued by one thread execute in issue order.
       for (int j = 0; ok && j < nb; ++j) {
         const int b = j & 1, s = j % NS;
-        if (j >= 2 && !wait_all1(&bars->pv_done[b], (uint32_t)(((j - 2) >> 1) & 1), abort_flag, pb.err)) {
-          ok = false;
-          break;
-        }
         if (!wait_all1(&bars->k_full[s], (uint32_t)((j / NS) & 1), abort_flag, pb.err)) {
           ok = false;
           break;
@@ -300,7 +299,7 @@ __global__ void __launch_bounds__(192, 1)
           // 16 bf16 = 32 bytes inside a 128-byte row; 64-column tiles apart
           const uint32_t offq = ((ks >> 2) * BM * 128 + (ks & 3) * 32) >> 4;
           const uint32_t offk = ((ks >> 2) * BN * 128 + (ks & 3) * 32) >> 4;
-          ptx::umma_ss_elect(tS[b], dq0 + offq, dk + offk, idesc_qk, ks > 0 ? 1u : 0u);
+          ptx::umma_ss_elect(b ? tS1 : tS0, dq0 + offq, dk + offk, idesc_qk, ks > 0 ? 1u : 0u);
         }
         ptx::umma_commit_elect(&bars->s_full[b]);
         ptx::umma_commit_elect(&bars->k_empty[s]);
@@ -333,15 +332,10 @@ __global__ void __launch_bounds__(192, 1)
       ptx::tc_fence_after();
       const uint32_t tS = lane_base + (b ? S::kColS1 : S::kColS0);
       float x[BN];
-      {
-        uint32_t r[BN];
 #pragma unroll
-        for (int cc = 0; cc < BN / 32; ++cc)
-          ptx::tmem_ld32(tS + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[cc * 32]));
-        ptx::tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < BN; ++i) x[i] = __uint_as_float(r[i]) * scale_log2;
-      }
+      for (int cc = 0; cc < BN / 32; ++cc)
+        ptx::tmem_ld32(tS + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&x[cc * 32]));
+      ptx::tmem_ld_wait();
       // visible keys of this row in this block: the first `lim` columns
       const bool ctx = j < n_ctx;
       int lim;
@@ -352,12 +346,22 @@ __global__ void __launch_bounds__(192, 1)
         const int end = pb.causal ? min(tile.q_len, rn + 1) : tile.q_len;
         lim = max(0, min(BN, end - kn0));
       }
-      float mx = -INFINITY;
+      if (__any_sync(0xffffffffu, lim < BN)) {
 #pragma unroll
-      for (int i = 0; i < BN; ++i) {
-        if (i >= lim) x[i] = -INFINITY;
-        mx = fmaxf(mx, x[i]);
+        for (int i = 0; i < BN; ++i) x[i] = i < lim ? x[i] : -INFINITY;
       }
+      // row max of the raw scores (scale > 0): 4 chains of 3-input max
+      float mq[4] = {x[0], x[1], x[2], x[3]};
+#pragma unroll
+      for (int i = 4; i < BN; i += 8) {
+        mq[0] = ptx::fmax3(mq[0], x[i], x[i + 1]);
+        mq[1] = ptx::fmax3(mq[1], x[i + 2], x[i + 3]);
+        if (i + 4 < BN) {
+          mq[2] = ptx::fmax3(mq[2], x[i + 4], x[i + 5]);
+          mq[3] = ptx::fmax3(mq[3], x[i + 6], x[i + 7]);
+        }
+      }
+      const float mx = ptx::fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * scale_log2;
       const float m_new = fmaxf(m, mx);
       const bool need = m == -INFINITY ? false : (m_new > m + kRescaleThreshold);
       float alpha = 1.f;
@@ -386,20 +390,29 @@ __global__ void __launch_bounds__(192, 1)
       } else if (m == -INFINITY) {
         m = m_new;
       }
-      const float m_use = m == -INFINITY ? 0.f : m;
-      float sum = 0.f;
+      const float neg_m = m == -INFINITY ? 0.f : -m;
+      const uint64_t scale2 = ptx::f2_pack(scale_log2, scale_log2);
+      const uint64_t negm2 = ptx::f2_pack(neg_m, neg_m);
+      uint64_t sp2[4] = {0, 0, 0, 0};   // packed partial sums
 #pragma unroll
       for (int cc = 0; cc < BN / 64; ++cc) {
         uint32_t r[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float p0 = ptx::ex2(x[cc * 64 + 2 * i] - m_use);
-          const float p1 = ptx::ex2(x[cc * 64 + 2 * i + 1] - m_use);
-          sum += p0 + p1;
+          float a0, a1;
+          ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(x[cc * 64 + 2 * i], x[cc * 64 + 2 * i + 1]), scale2, negm2), a0, a1);
+          const uint64_t pp = ptx::f2_pack(ptx::ex2(a0), ptx::ex2(a1));
+          sp2[i & 3] = ptx::f2_add(sp2[i & 3], pp);
+          float p0, p1;
+          ptx::f2_unpack(pp, p0, p1);
           r[i] = ptx::pack_bf16(p0, p1);
         }
         ptx::tmem_st32(tS + cc * 32, r);
       }
+      float spf[8];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) ptx::f2_unpack(sp2[k], spf[2 * k], spf[2 * k + 1]);
+      const float sum = ((spf[0] + spf[1]) + (spf[2] + spf[3])) + ((spf[4] + spf[5]) + (spf[6] + spf[7]));
       ptx::tmem_st_wait();
       l = l * alpha + sum;
       ptx::tc_fence_before();

@@ -7,6 +7,7 @@
 // shape (decode: one new token; prefill / chunked prefill: many), and the
 // per-kernel work lists are built on the host, uploaded with one copy and
 // consumed by the kernels.
+#include <cmath>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
@@ -419,6 +420,8 @@ extern "C" RPA_API int rpa_forward(const void *q, const void *k_new, const void 
                            float scale, int32_t causal, void *out, float *lse,
                            const rpa_dims *dims, void *stream_ptr) {
   cudaStream_t stream = (cudaStream_t)stream_ptr;
+  // the kernels take row maxima of the raw scores: the scale must be > 0
+  if (!(scale > 0.f) || !std::isfinite(scale)) return RPA_ERR_INVALID_ARG;
   try {
     HostPlan hp;
     int rc = plan_checked(cu_q_lens, kv_lens, num_seqs, distribution, dims, hp);

@@ -169,3 +169,21 @@ def test_forward_rejects_before_touching_device(rb):
                          ctypes.byref(d), None)
     assert rc == 3
     assert rb.rpa_status_string(3) == "invalid sequence lengths"
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.125, float("nan"), float("inf")])
+def test_forward_rejects_non_positive_scale(rb, scale):
+    """The scale must be positive and finite (the kernels take row maxima of
+    the unscaled scores); anything else is rejected before device work."""
+    lib = rb.library()
+    cu = np.array([0, 1], np.int32)
+    kv = np.array([4], np.int32)
+    d = dims(total_q_tokens=1)
+    fake = ctypes.c_void_p(0x1000)
+    rc = lib.rpa_forward(fake, fake, fake, fake, fake, fake, cu.ctypes.data_as(ctypes.c_void_p),
+                         kv.ctypes.data_as(ctypes.c_void_p), 1, None, ctypes.c_float(scale), 1, fake, None,
+                         ctypes.byref(d), None)
+    assert rc == 1
+    rc = lib.rpa_decode_noalloc(fake, fake, fake, fake, fake, fake, kv.ctypes.data_as(ctypes.c_void_p), 1,
+                                ctypes.c_float(scale), fake, None, ctypes.byref(d), None, None)
+    assert rc == 1
