@@ -10,9 +10,11 @@
 //              (tcgen05.ld), P goes back into TMEM as bf16 (tcgen05.st),
 //              online softmax in log2 units with a lazily refreshed running
 //              max (O is rescaled only when the max grows by more than 2^8);
-//              epilogue O / l -> bf16, lse; then the tile's share of the
-//              new K/V rows is copied into its cache pages.
-//   warp 4     producer: TMA of the Q tile, then K and V blocks of BN keys:
+//              epilogue O / l -> bf16, lse.  Before the first block (while
+//              Q and the first S are on their way) they copy the tile's
+//              share of the new K/V rows into its cache pages.
+//   warp 4     producer: TMA of the Q tile, then K and V blocks of BN keys
+//              into rings of their own (K as soon as its stage is free):
 //              cached context from the pages (one box per page segment),
 //              new tokens from k_new / v_new.  Rows of a block that hold no
 //              valid key (past the context, past the sequence, bad pages)
@@ -45,11 +47,14 @@ template <int D>
 struct PrefillShape {
   static constexpr int BM = kPrefillTileRows;          // 128 query rows
   static constexpr int BN = D == 256 ? 64 : 128;       // keys per block
-  static constexpr int NS = 2;                         // K/V stages
+  // K and V rings of their own: a block's K is needed first (QK(j) comes
+  // before PV(j-1)), its V a softmax later
+  static constexpr int NSK = 3;                        // K stages
+  static constexpr int NSV = 2;                        // V stages
   static constexpr int kHalves = D / 64;
   static constexpr int kQBytes = kHalves * BM * 128;
   static constexpr int kKVBytes = kHalves * BN * 128;  // one K or one V block
-  static constexpr int kData = kQBytes + 2 * NS * kKVBytes;
+  static constexpr int kData = kQBytes + (NSK + NSV) * kKVBytes;
   static constexpr int kBarriers = 32;
   // at least 116 KB so that two CTAs never share an SM (each owns all 512
   // TMEM columns)
@@ -62,7 +67,7 @@ struct PrefillShape {
 
 struct Bars {
   uint64_t q_full;
-  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t k_full[3], k_empty[3], v_full[2], v_empty[2];
   uint64_t s_full[2], p_full[2], pv_done[2];
   uint64_t fix, drain;
 };
@@ -95,12 +100,12 @@ __global__ void __launch_bounds__(192, 1)
                    const __grid_constant__ CUtensorMap tm_vn, const Problem pb,
                    const PrefillTile *__restrict__ tiles, float scale_log2) {
   using S = PrefillShape<D>;
-  constexpr int BM = S::BM, BN = S::BN, NS = S::NS;
+  constexpr int BM = S::BM, BN = S::BN, NSK = S::NSK, NSV = S::NSV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sQ = base;
-  uint8_t *sK = sQ + S::kQBytes;                 // NS blocks
-  uint8_t *sV = sK + NS * S::kKVBytes;           // NS blocks
+  uint8_t *sK = sQ + S::kQBytes;                 // NSK blocks
+  uint8_t *sV = sK + NSK * S::kKVBytes;          // NSV blocks
   Bars *bars = reinterpret_cast<Bars *>(base + S::kData);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -121,9 +126,11 @@ __global__ void __launch_bounds__(192, 1)
 
   if (tid == 0) {
     ptx::mbar_init(&bars->q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NSK; ++i) {
       ptx::mbar_init(&bars->k_full[i], 1);
       ptx::mbar_init(&bars->k_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&bars->v_full[i], 1);
       ptx::mbar_init(&bars->v_empty[i], 1);
       ptx::mbar_init(&bars->s_full[i], 1);
@@ -156,15 +163,16 @@ __global__ void __launch_bounds__(192, 1)
     const int br = pb.p < BN ? pb.p : BN;      // rows per page-segment box
     const int nseg = BN / br;                  // <= 16
     uint32_t fix_phase = 0;
-    int issued = 0;                            // blocks whose copies were queued
+    int gk = 0, gv = 0;                        // blocks whose K (V) copies were queued and published
+    bool fix_pending = false;
     ptx::mbar_arrive_expect_tx_elect(&bars->q_full, S::kQBytes);
     for (int hh = 0; hh < S::kHalves; ++hh)
       ptx::tma_load_3d_elect(sQ + hh * BM * 128, &tm_q, &bars->q_full, hh * 64, h, tile.q_start + r0);
     for (int j = 0; j < nb; ++j) {
-      const int s = j % NS;
-      const uint32_t ph = (uint32_t)((j / NS) & 1);
-      uint8_t *dk = sK + s * S::kKVBytes;
-      uint8_t *dv = sV + s * S::kKVBytes;
+      const int sk = j % NSK, sv = j % NSV;
+      const uint32_t phk = (uint32_t)((j / NSK) & 1), phv = (uint32_t)((j / NSV) & 1);
+      uint8_t *dk = sK + sk * S::kKVBytes;
+      uint8_t *dv = sV + sv * S::kKVBytes;
       // Block geometry: valid rows; for context blocks the page of each
       // segment (lane sg reads segment sg's page-table entry).
       const bool ctx = j < n_ctx;
@@ -189,72 +197,80 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t seg_bytes = (uint32_t)(S::kHalves * br * 128);
       const uint32_t blk_bytes = ctx ? (uint32_t)__popc(loaded_mask) * seg_bytes : (uint32_t)S::kKVBytes;
 
-      if (j >= NS) {
-        if (!wait_all1(&bars->k_empty[s], ph ^ 1u, abort_flag, pb.err)) break;
-        if (!wait_all1(&bars->v_empty[s], ph ^ 1u, abort_flag, pb.err)) break;
+      // the copies of one operand (K or V) of this block into dst
+      auto load = [&](uint8_t *dst, const CUtensorMap *tm_new, const CUtensorMap *tm_ctx, uint64_t *bar) {
+        if (!ctx) {
+          const int row = tile.q_start + pos0;
+          for (int hh = 0; hh < S::kHalves; ++hh)
+            ptx::tma_load_3d_elect(dst + hh * BN * 128, tm_new, bar, hh * 64, hk, row);
+        } else {
+          // every lane takes part in the broadcast of segment sg's page id
+          for (int sg = 0; sg < nseg; ++sg) {
+            const int pg = __shfl_sync(0xffffffffu, page, sg);
+            if (!((loaded_mask >> sg) & 1u)) continue;
+            const int sp = pos0 + sg * br;
+            const int row = pg * pb.p + (sp % pb.p);
+            for (int hh = 0; hh < S::kHalves; ++hh)
+              ptx::tma_load_3d_elect(dst + hh * BN * 128 + sg * br * 128, tm_ctx, bar, hh * 64, hk, row);
+          }
+        }
+      };
+      if (!fix) {
+        // K as soon as its stage is free, then V
+        if (j >= NSK && !wait_all1(&bars->k_empty[sk], phk ^ 1u, abort_flag, pb.err)) break;
+        ptx::mbar_arrive_expect_tx_elect(&bars->k_full[sk], blk_bytes);
+        load(dk, &tm_kn, &tm_kc, &bars->k_full[sk]);
+        ++gk;
+        if (j >= NSV && !wait_all1(&bars->v_empty[sv], phv ^ 1u, abort_flag, pb.err)) break;
+        ptx::mbar_arrive_expect_tx_elect(&bars->v_full[sv], blk_bytes);
+        load(dv, &tm_vn, &tm_vc, &bars->v_full[sv]);
+        ++gv;
+        continue;
       }
-      uint64_t *kb = fix ? &bars->fix : &bars->k_full[s];
-      uint64_t *vb = fix ? &bars->fix : &bars->v_full[s];
-      if (fix) {
-        ptx::mbar_arrive_expect_tx_elect(&bars->fix, 2 * blk_bytes);
-      } else {
-        ptx::mbar_arrive_expect_tx_elect(&bars->k_full[s], blk_bytes);
-        ptx::mbar_arrive_expect_tx_elect(&bars->v_full[s], blk_bytes);
+      // Partial block or bad pages: both operands through the private
+      // barrier (it completes even with no copies: the arrival carried zero
+      // expected bytes), zero every row that holds no valid key, publish.
+      if ((j >= NSK && !wait_all1(&bars->k_empty[sk], phk ^ 1u, abort_flag, pb.err)) ||
+          (j >= NSV && !wait_all1(&bars->v_empty[sv], phv ^ 1u, abort_flag, pb.err)))
+        break;
+      ptx::mbar_arrive_expect_tx_elect(&bars->fix, 2 * blk_bytes);
+      load(dk, &tm_kn, &tm_kc, &bars->fix);
+      load(dv, &tm_vn, &tm_vc, &bars->fix);
+      const bool fok = wait_all1(&bars->fix, fix_phase, abort_flag, pb.err);
+      fix_phase ^= 1u;
+      if (!fok) {
+        fix_pending = true;   // copies may still be in flight: drained below
+        break;
       }
-      if (!ctx) {
-        const int row = tile.q_start + pos0;
+      for (int r = lane; r < BN; r += 32) {
+        const bool bad_row = r >= valid || (ctx && !((loaded_mask >> (r / br)) & 1u));
+        if (!bad_row) continue;
         for (int hh = 0; hh < S::kHalves; ++hh) {
-          ptx::tma_load_3d_elect(dk + hh * BN * 128, &tm_kn, kb, hh * 64, hk, row);
-          ptx::tma_load_3d_elect(dv + hh * BN * 128, &tm_vn, vb, hh * 64, hk, row);
-        }
-      } else {
-        // every lane takes part in the broadcast of segment sg's page id
-        for (int sg = 0; sg < nseg; ++sg) {
-          const int pg = __shfl_sync(0xffffffffu, page, sg);
-          if (!((loaded_mask >> sg) & 1u)) continue;
-          const int sp = pos0 + sg * br;
-          const int row = pg * pb.p + (sp % pb.p);
-          for (int hh = 0; hh < S::kHalves; ++hh) {
-            ptx::tma_load_3d_elect(dk + hh * BN * 128 + sg * br * 128, &tm_kc, kb, hh * 64, hk, row);
-            ptx::tma_load_3d_elect(dv + hh * BN * 128 + sg * br * 128, &tm_vc, vb, hh * 64, hk, row);
-          }
-        }
-      }
-      ++issued;
-      if (fix) {
-        // Wait for this block's copies (the private barrier completes even
-        // with no copies: the arrival carried zero expected bytes), zero
-        // every row that holds no valid key, then publish the block.
-        const bool ok = wait_all1(&bars->fix, fix_phase, abort_flag, pb.err);
-        fix_phase ^= 1u;
-        if (!ok) break;
-        for (int r = lane; r < BN; r += 32) {
-          const bool bad_row = r >= valid || (ctx && !((loaded_mask >> (r / br)) & 1u));
-          if (!bad_row) continue;
-          for (int hh = 0; hh < S::kHalves; ++hh) {
-            uint4 *pk = reinterpret_cast<uint4 *>(dk + hh * BN * 128 + r * 128);
-            uint4 *pv = reinterpret_cast<uint4 *>(dv + hh * BN * 128 + r * 128);
+          uint4 *pk = reinterpret_cast<uint4 *>(dk + hh * BN * 128 + r * 128);
+          uint4 *pv = reinterpret_cast<uint4 *>(dv + hh * BN * 128 + r * 128);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              pk[q] = make_uint4(0, 0, 0, 0);
-              pv[q] = make_uint4(0, 0, 0, 0);
-            }
+          for (int q = 0; q < 8; ++q) {
+            pk[q] = make_uint4(0, 0, 0, 0);
+            pv[q] = make_uint4(0, 0, 0, 0);
           }
         }
-        ptx::fence_proxy_async_smem();
-        __syncwarp();
-        ptx::mbar_arrive_elect(&bars->k_full[s]);
-        ptx::mbar_arrive_elect(&bars->v_full[s]);
       }
+      ptx::fence_proxy_async_smem();
+      __syncwarp();
+      ptx::mbar_arrive_elect(&bars->k_full[sk]);
+      ptx::mbar_arrive_elect(&bars->v_full[sv]);
+      ++gk;
+      ++gv;
     }
     // Before the CTA can end, every copy this warp queued must have landed
     // (bounded waits; they complete without any other warp).
     if (lane == 0) {
       ptx::mbar_wait(&bars->q_full, 0);
-      for (int j = issued - NS < 0 ? 0 : issued - NS; j < issued; ++j) {
-        ptx::mbar_wait(&bars->k_full[j % NS], (uint32_t)((j / NS) & 1));
-        ptx::mbar_wait(&bars->v_full[j % NS], (uint32_t)((j / NS) & 1));
-      }
+      for (int j = gk - NSK < 0 ? 0 : gk - NSK; j < gk; ++j)
+        ptx::mbar_wait(&bars->k_full[j % NSK], (uint32_t)((j / NSK) & 1));
+      for (int j = gv - NSV < 0 ? 0 : gv - NSV; j < gv; ++j)
+        ptx::mbar_wait(&bars->v_full[j % NSV], (uint32_t)((j / NSV) & 1));
+      if (fix_pending) ptx::mbar_wait(&bars->fix, fix_phase ^ 1u);
     }
     __syncwarp();
   } else if (warp == 5) {
@@ -270,9 +286,9 @@ __global__ void __launch_bounds__(192, 1)
       const uint64_t dv0 = ptx::umma_desc_sw128(ptx::smem_u32(sV), BN * 128, 1024);
       bool ok = wait_all1(&bars->q_full, 0, abort_flag, pb.err);
       auto pv = [&](int i) -> bool {
-        const int b = i & 1, s = i % NS;
+        const int b = i & 1, s = i % NSV;
         if (!wait_all1(&bars->p_full[b], (uint32_t)((i >> 1) & 1), abort_flag, pb.err)) return false;
-        if (!wait_all1(&bars->v_full[s], (uint32_t)((i / NS) & 1), abort_flag, pb.err)) return false;
+        if (!wait_all1(&bars->v_full[s], (uint32_t)((i / NSV) & 1), abort_flag, pb.err)) return false;
         ptx::tc_fence_after();
         const uint64_t dv = dv0 + (uint64_t)((s * S::kKVBytes) >> 4);
 #pragma unroll
@@ -287,8 +303,8 @@ __global__ void __launch_bounds__(192, 1)
       // after PV(j-2) without waiting for it to finish, because tcgen05.mma
       // operations issued by one thread execute in issue order.
       for (int j = 0; ok && j < nb; ++j) {
-        const int b = j & 1, s = j % NS;
-        if (!wait_all1(&bars->k_full[s], (uint32_t)((j / NS) & 1), abort_flag, pb.err)) {
+        const int b = j & 1, s = j % NSK;
+        if (!wait_all1(&bars->k_full[s], (uint32_t)((j / NSK) & 1), abort_flag, pb.err)) {
           ok = false;
           break;
         }
@@ -319,6 +335,32 @@ __global__ void __launch_bounds__(192, 1)
     const int row = tid;                           // 0..127 == TMEM lane
     const int rn = r0 + row;                       // new-token index of this row
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    // Fused cache update, first: the softmax warps would otherwise wait for
+    // Q and the first S.  The G CTAs of this KV head split the tile's new
+    // rows between them; each row's K and V are copied into its page slot.
+    {
+      const int g = h % G;
+      const int ra = (g * tile.rows) / G, rb = ((g + 1) * tile.rows) / G;
+      const int chunks = D / 8;   // 16-byte chunks per row
+      const __nv_bfloat16 *kn = reinterpret_cast<const __nv_bfloat16 *>(pb.k_new);
+      const __nv_bfloat16 *vn = reinterpret_cast<const __nv_bfloat16 *>(pb.v_new);
+      __nv_bfloat16 *kc = reinterpret_cast<__nv_bfloat16 *>(pb.k_cache);
+      __nv_bfloat16 *vc = reinterpret_cast<__nv_bfloat16 *>(pb.v_cache);
+      for (int idx = tid; idx < (rb - ra) * chunks; idx += 128) {
+        const int r = ra + idx / chunks, ch = idx % chunks;
+        const int i = r0 + r;                  // new-token index
+        const int pos = c + i;
+        const int pg = pt_row[pos / pb.p];
+        if (pg < 0 || pg >= pb.num_pages) {
+          if (ch == 0) atomicOr(pb.err, RPA_DEV_BAD_PAGE);
+          continue;
+        }
+        const size_t src = ((size_t)(tile.q_start + i) * pb.hkv + hk) * D + ch * 8;
+        const size_t dst = (((size_t)pg * pb.p + pos % pb.p) * pb.hkv + hk) * D + ch * 8;
+        *reinterpret_cast<uint4 *>(kc + dst) = *reinterpret_cast<const uint4 *>(kn + src);
+        *reinterpret_cast<uint4 *>(vc + dst) = *reinterpret_cast<const uint4 *>(vn + src);
+      }
+    }
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nb; ++j) {
@@ -442,31 +484,6 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       if (store && pb.lse != nullptr) pb.lse[(size_t)(tile.q_start + rn) * pb.hq + h] = (m + log2f(l)) * kLn2;
-    }
-    // Fused cache update: the G CTAs of this KV head split the tile's new
-    // rows between them; each row's K and V are copied into its page slot.
-    {
-      const int g = h % G;
-      const int ra = (g * tile.rows) / G, rb = ((g + 1) * tile.rows) / G;
-      const int chunks = D / 8;   // 16-byte chunks per row
-      const __nv_bfloat16 *kn = reinterpret_cast<const __nv_bfloat16 *>(pb.k_new);
-      const __nv_bfloat16 *vn = reinterpret_cast<const __nv_bfloat16 *>(pb.v_new);
-      __nv_bfloat16 *kc = reinterpret_cast<__nv_bfloat16 *>(pb.k_cache);
-      __nv_bfloat16 *vc = reinterpret_cast<__nv_bfloat16 *>(pb.v_cache);
-      for (int idx = tid; idx < (rb - ra) * chunks; idx += 128) {
-        const int r = ra + idx / chunks, ch = idx % chunks;
-        const int i = r0 + r;                  // new-token index
-        const int pos = c + i;
-        const int pg = pt_row[pos / pb.p];
-        if (pg < 0 || pg >= pb.num_pages) {
-          if (ch == 0) atomicOr(pb.err, RPA_DEV_BAD_PAGE);
-          continue;
-        }
-        const size_t src = ((size_t)(tile.q_start + i) * pb.hkv + hk) * D + ch * 8;
-        const size_t dst = (((size_t)pg * pb.p + pos % pb.p) * pb.hkv + hk) * D + ch * 8;
-        *reinterpret_cast<uint4 *>(kc + dst) = *reinterpret_cast<const uint4 *>(kn + src);
-        *reinterpret_cast<uint4 *>(vc + dst) = *reinterpret_cast<const uint4 *>(vn + src);
-      }
     }
   }
 
