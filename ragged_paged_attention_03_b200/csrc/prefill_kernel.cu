@@ -346,19 +346,39 @@ __global__ void __launch_bounds__(192, 1)
       const __nv_bfloat16 *vn = reinterpret_cast<const __nv_bfloat16 *>(pb.v_new);
       __nv_bfloat16 *kc = reinterpret_cast<__nv_bfloat16 *>(pb.k_cache);
       __nv_bfloat16 *vc = reinterpret_cast<__nv_bfloat16 *>(pb.v_cache);
-      for (int idx = tid; idx < (rb - ra) * chunks; idx += 128) {
-        const int r = ra + idx / chunks, ch = idx % chunks;
-        const int i = r0 + r;                  // new-token index
-        const int pos = c + i;
-        const int pg = pt_row[pos / pb.p];
-        if (pg < 0 || pg >= pb.num_pages) {
-          if (ch == 0) atomicOr(pb.err, RPA_DEV_BAD_PAGE);
-          continue;
+      // kBatch chunks per thread in flight: the loads (sources and page-table
+      // entries) of a batch are issued before its stores
+      constexpr int kBatch = 8;
+      const int total = (rb - ra) * chunks;
+      for (int base = tid; base < total; base += 128 * kBatch) {
+        uint4 kq[kBatch], vq[kBatch];
+        int pgq[kBatch];
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+          const int idx = base + q * 128;
+          if (idx < total) {
+            const int i = r0 + ra + idx / chunks;   // new-token index
+            const size_t src = ((size_t)(tile.q_start + i) * pb.hkv + hk) * D + (idx % chunks) * 8;
+            kq[q] = *reinterpret_cast<const uint4 *>(kn + src);
+            vq[q] = *reinterpret_cast<const uint4 *>(vn + src);
+            pgq[q] = pt_row[(c + i) / pb.p];
+          }
         }
-        const size_t src = ((size_t)(tile.q_start + i) * pb.hkv + hk) * D + ch * 8;
-        const size_t dst = (((size_t)pg * pb.p + pos % pb.p) * pb.hkv + hk) * D + ch * 8;
-        *reinterpret_cast<uint4 *>(kc + dst) = *reinterpret_cast<const uint4 *>(kn + src);
-        *reinterpret_cast<uint4 *>(vc + dst) = *reinterpret_cast<const uint4 *>(vn + src);
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+          const int idx = base + q * 128;
+          if (idx >= total) continue;
+          const int i = r0 + ra + idx / chunks, ch = idx % chunks;
+          const int pos = c + i;
+          const int pg = pgq[q];
+          if (pg < 0 || pg >= pb.num_pages) {
+            if (ch == 0) atomicOr(pb.err, RPA_DEV_BAD_PAGE);
+            continue;
+          }
+          const size_t dst = (((size_t)pg * pb.p + pos % pb.p) * pb.hkv + hk) * D + ch * 8;
+          *reinterpret_cast<uint4 *>(kc + dst) = kq[q];
+          *reinterpret_cast<uint4 *>(vc + dst) = vq[q];
+        }
       }
     }
     float m = -INFINITY, l = 0.f;
