@@ -48,6 +48,8 @@ WORKLOAD_TEXT = {
                     "log-U[1024,8192] context, Hq 32 / Hkv 8, D 128, page 16, bf16, causal",
     "long_d256": "long context: 32 decode seqs kv 131072 + 4 prefill seqs 4096, Hq 16 / Hkv 4, "
                  "D 256, page 64, bf16, causal",
+    "prefill_4x4096_d256": "prefill: 4 fresh seqs q_len = kv_len = 4096, Hq 16 / Hkv 4, D 256, page 64, "
+                           "bf16, N(0,1), shuffled 1.25x pool (the prefill rows of the long-context batch)",
 }
 
 
@@ -361,7 +363,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workloads", default="decode_128,prefill_8x2048,prefill_8x2048:noncausal,"
-                                           "mixed_96d_4c,long_d256")
+                                           "mixed_96d_4c,long_d256,prefill_4x4096_d256")
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the cpu_baseline sample")
     ap.add_argument("--max-seqs", type=int, default=None,

@@ -125,6 +125,8 @@ def _lengths(name: str, gen: torch.Generator):
         return [1] * 96 + [512] * 4, dec + [p + 512 for p in prior]
     if name == "long_d256":
         return [1] * 32 + [4096] * 4, [131072] * 32 + [4096] * 4
+    if name == "prefill_4x4096_d256":
+        return [4096] * 4, [4096] * 4
     raise KeyError(name)
 
 
@@ -135,6 +137,8 @@ WORKLOADS = {
     "prefill_8x2048": (BF16, 32, 8, 128, 16, True, 1.0, 3, 1.25),
     "mixed_96d_4c": (BF16, 32, 8, 128, 16, True, 1.0, 4, 1.25),
     "long_d256": (BF16, 16, 4, 256, 64, True, 1.0, 5, 1.25),
+    # the prefill sequences of long_d256 alone (a size a profiler capture fits)
+    "prefill_4x4096_d256": (BF16, 16, 4, 256, 64, True, 1.0, 6, 1.25),
 }
 
 
