@@ -142,6 +142,38 @@ def test_chunked_prefill_long_context(oracle_mod, loaders):
         binding.rpa_set_option(binding.RPA_OPT_PREFILL_LOADERS, old)
 
 
+MORE = [
+    # chunked prefill after a cache, both prefill builds forced below: page 8 and 256, D 64 / 128
+    ([300, 1, 129], [1500, 4000, 700], 16, 4, 64, 8, True),
+    ([257, 64, 1], [3000, 64, 9000], 32, 8, 128, 256, True),
+    ([200, 17], [2600, 900], 8, 8, 128, 32, False),
+    # head_dim 256: chunked rows after context, ragged tails, page 64 and 16
+    ([130, 3, 1], [1000, 260, 5000], 16, 4, 256, 64, True),
+    ([65, 1], [65, 300], 8, 2, 256, 16, False),
+    # decode: G = 1 and G = 16 (two 8-head groups per tile), long and short mixed
+    ([1] * 6, [1, 2, 4096, 5000, 31, 12000], 8, 8, 128, 16, True),
+    ([1] * 4, [9000, 17, 3000, 128], 32, 2, 128, 16, True),
+    ([1] * 5, [1, 777, 8000, 64, 20000], 16, 1, 64, 32, True),
+]
+
+
+@pytest.mark.parametrize("loaders", [0, 2])
+@pytest.mark.parametrize("case", range(len(MORE)))
+def test_more_shapes(oracle_mod, case, loaders):
+    """Page sizes, head dims, GQA ratios and length mixes beyond the small
+    set, with the prefill kernel build chosen by the planner (0) or the one
+    producer warp per operand build forced (2)."""
+    from ragged_paged_attention_03_b200 import binding
+    ql, kv, hq, hkv, d, p, causal = MORE[case]
+    old = binding.rpa_set_option(binding.RPA_OPT_PREFILL_LOADERS, loaders)
+    try:
+        prob = I.make_problem(ql, kv, num_q_heads=hq, num_kv_heads=hkv, head_dim=d, page_size=p,
+                              dtype=I.BF16, causal=causal, seed=500 + case, pool=1.3)
+        full_check(oracle_mod, prob)
+    finally:
+        binding.rpa_set_option(binding.RPA_OPT_PREFILL_LOADERS, old)
+
+
 def test_bad_page_is_flagged_not_read(oracle_mod):
     """A page-table entry outside the pool is reported through the device
     error word; the kernels never dereference it."""
