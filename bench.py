@@ -262,12 +262,14 @@ def value_of(name, work, ms, n):
     return n * work["tokens"] / (ms * 1e-3)
 
 
-def roofline(name, work, kern, pk):
-    """The dominant kernel of the step against its own roofline."""
+def roofline(name, work, kern, pk, steps):
+    """The dominant kernel class of the step against its own roofline: its
+    device time per step (a class may launch more than once per step, e.g.
+    decode for long and for packed short sequences)."""
     launches = {k: v for k, v in kern.items() if v[0] > 0}
     top = max(launches, key=lambda k: launches[k][1])
     n, total_ms = launches[top]
-    avg_s = total_ms / n * 1e-3
+    avg_s = total_ms / steps * 1e-3
     if top == "prefill":
         achieved = work["prefill_flops"] / avg_s / 1e12
         r = {"bound": "tensor", "achieved": achieved, "peak": pk["tc"], "unit": "TFLOP/s",
@@ -279,7 +281,8 @@ def roofline(name, work, kern, pk):
              "peak_source": f"{pk['source']} HBM copy"}
     r["frac"] = r["achieved"] / r["peak"]
     r["kernel"] = top
-    r["kernel_ms"] = total_ms / n
+    r["kernel_ms"] = total_ms / steps
+    r["kernel_launches_per_step"] = n / steps
     r["traffic"] = traffic_for(top, name)
     r["kernel_share"] = {k: round(v[1] / sum(x[1] for x in launches.values()), 4)
                          for k, v in launches.items()}
@@ -441,7 +444,7 @@ def main():
                            "l2": "flushed between steps (256 MiB write)",
                            "tokens": work["tokens"], "bytes": work["bytes"],
                            "flops": work["flops"]},
-                "roofline": roofline(name, work, kern, pk),
+                "roofline": roofline(name, work, kern, pk, args.steps),
                 "e2e": {"value": value_of(name, work, e2e_ms, n), "unit": unit,
                         "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},

@@ -161,6 +161,9 @@ typedef struct {
   int32_t combine_rows;      /* decode sequences that need the LSE combine */
   int32_t prefill_tiles;     /* (sequence, query tile) work items, per Q head */
   int64_t plan_bytes;        /* bytes of the plan copied to the device */
+  int32_t decode_packed;     /* of decode_items: short whole sequences run
+                                four per CTA, one per warp */
+  int32_t pad;
 } rpa_plan_info;
 
 /*
@@ -188,12 +191,19 @@ enum {
                                       mixed batch concurrently on two streams
                                       (default 0: one after the other, faster
                                       on the measured mixes) */
-  RPA_OPT_PREFILL_LOADERS = 5      /* TMA producer warps of the head_dim <= 128
+  RPA_OPT_PREFILL_LOADERS = 5,     /* TMA producer warps of the head_dim <= 128
                                       prefill kernel: 1 (K and V share one), 2
                                       (one each; the cache update gets one warp
                                       instead of two), 0 = chosen per batch:
                                       2 when the prefill rows' cached context
                                       outnumbers their new tokens (default 0) */
+  RPA_OPT_DECODE_PACK_BLOCKS = 6   /* decode sequences of at most this many
+                                      16-token blocks (and within one work
+                                      item) run four per CTA, one per warp,
+                                      when they make at least 296 such CTAs
+                                      (two per SM); fewer stay in the main
+                                      decode launch (default 64; 0 restores
+                                      it, < 0: never) */
 };
 RPA_API int64_t rpa_set_option(int32_t option, int64_t value);
 

@@ -29,6 +29,7 @@ RPA_OPT_DISABLE_PREFILL_TC = 2
 RPA_OPT_PREFILL_SMS = 3
 RPA_OPT_CONCURRENT_MIXED = 4
 RPA_OPT_PREFILL_LOADERS = 5
+RPA_OPT_DECODE_PACK_BLOCKS = 6
 
 
 class rpa_dims(ctypes.Structure):
@@ -40,7 +41,8 @@ class rpa_dims(ctypes.Structure):
 class rpa_plan_info(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "num_decode", "num_prefill", "num_generic", "num_empty", "decode_items",
-        "decode_max_splits", "combine_rows", "prefill_tiles")] + [("plan_bytes", ctypes.c_int64)]
+        "decode_max_splits", "combine_rows", "prefill_tiles")] + [("plan_bytes", ctypes.c_int64)] + [
+        ("decode_packed", ctypes.c_int32), ("pad", ctypes.c_int32)]
 
 
 class RpaError(RuntimeError):

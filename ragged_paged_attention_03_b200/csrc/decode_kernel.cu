@@ -8,6 +8,9 @@
 // * One CTA per (work item, KV head).  A work item is a chunk of 16-token
 //   blocks of one sequence; long sequences are cut into several items whose
 //   partial results the combine kernel merges (log-sum-exp weighting).
+// * Short sequences are packed instead: four whole-sequence items per CTA,
+//   one per warp, each warp streaming all of its item's blocks (the pages'
+//   fix for requests too short to fill the bandwidth on their own).
 // * The CTA's four warps stream disjoint blocks (block b goes to warp
 //   b mod 4), each with its own ring of shared-memory stages fed by TMA
 //   (cp.async.bulk.tensor, 128-byte swizzle, one 16-row box per page part
@@ -54,11 +57,14 @@ __device__ __forceinline__ uint32_t tile_off(int r, int ch) {
   return (uint32_t)((ch >> 3) * (16 * 128) + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
 }
 
-template <int D, int NG>
+// PACK: each warp takes a whole work item of its own (item blockIdx.x * 4 +
+// warp) -- short sequences, several per CTA -- and writes its result from
+// registers; otherwise the four warps share one item and merge at the end.
+template <int D, int NG, bool PACK>
 __global__ void __launch_bounds__(128) decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                                                      const __grid_constant__ CUtensorMap tm_v,
                                                      const Problem pb, const DecodeItem *__restrict__ items,
-                                                     float *__restrict__ part_o,
+                                                     int n_items, float *__restrict__ part_o,
                                                      float *__restrict__ part_lse, float scale_log2) {
   using S = DecodeShape<D>;
   constexpr int NST = S::kStages;
@@ -71,7 +77,10 @@ __global__ void __launch_bounds__(128) decode_kernel(const __grid_constant__ CUt
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const DecodeItem it = items[blockIdx.x];
+  const int item_idx = PACK ? (int)blockIdx.x * kWarps + warp : (int)blockIdx.x;
+  const bool has_item = item_idx < n_items;   // PACK: the last CTA may hold fewer items
+  DecodeItem it = items[has_item ? item_idx : 0];
+  if (!has_item) it.blk_begin = it.blk_end = 0;
   const int hk = blockIdx.y;
   const int G = pb.hq / pb.hkv;
   const int kv = it.kv_len;
@@ -80,20 +89,22 @@ __global__ void __launch_bounds__(128) decode_kernel(const __grid_constant__ CUt
   const int nblk_total = (kv + 15) >> 4;      // the last block holds position c
   const int first_page = (it.blk_begin * 16) / P;
   const int last_page = (min(it.blk_end * 16, kv) - 1) / P;
-  const int npg = last_page - first_page + 1;
+  const int npg = has_item ? last_page - first_page + 1 : 0;
   const int32_t *pt_row = pb.page_table + (size_t)it.seq * pb.max_pages;
+  // PACK: a quarter of the page slots per warp
+  int32_t *my_pages = pages + (PACK ? warp * (kMaxItemPages / kWarps) : 0);
 
   if (tid == 0) {
     ptx::tma_prefetch_desc(&tm_k);
     ptx::tma_prefetch_desc(&tm_v);
   }
-  for (int i = tid; i < npg; i += blockDim.x) {
+  for (int i = PACK ? lane : tid; i < npg; i += PACK ? 32 : (int)blockDim.x) {
     int pg = pt_row[first_page + i];
     if (pg < 0 || pg >= pb.num_pages) {
       atomicOr(pb.err, RPA_DEV_BAD_PAGE);
       pg = -1;
     }
-    pages[i] = pg;
+    my_pages[i] = pg;
   }
   if (tid < kWarps * NST) ptx::mbar_init(&bars[tid], 1);
   ptx::fence_barrier_init();
@@ -107,7 +118,7 @@ __global__ void __launch_bounds__(128) decode_kernel(const __grid_constant__ CUt
   // (lane 0 only).  Boxes holding no cached position are skipped; their rows
   // are filled when the block is consumed.
   auto issue = [&](int k) {
-    const int b = it.blk_begin + warp + kWarps * k;
+    const int b = it.blk_begin + (PACK ? k : warp + kWarps * k);
     if (b >= it.blk_end) return;
     const int st = k % NST;
     uint8_t *sk = my_ring + st * S::kStage;
@@ -115,7 +126,7 @@ __global__ void __launch_bounds__(128) decode_kernel(const __grid_constant__ CUt
     uint32_t bytes = 0;
     for (int r0 = 0; r0 < 16; r0 += box_rows) {
       const int pos = b * 16 + r0;
-      if (pos < c && pages[pos / P - first_page] >= 0) bytes += 2u * S::kHalves * 128u * box_rows;
+      if (pos < c && my_pages[pos / P - first_page] >= 0) bytes += 2u * S::kHalves * 128u * box_rows;
     }
     if (bytes == 0) {
       ptx::mbar_arrive(&my_bars[st]);
@@ -125,7 +136,7 @@ __global__ void __launch_bounds__(128) decode_kernel(const __grid_constant__ CUt
     for (int r0 = 0; r0 < 16; r0 += box_rows) {
       const int pos = b * 16 + r0;
       if (pos >= c) break;
-      const int pg = pages[pos / P - first_page];
+      const int pg = my_pages[pos / P - first_page];
       if (pg < 0) continue;
       const int row = pg * P + (pos % P);
 #pragma unroll
@@ -178,7 +189,7 @@ __global__ void __launch_bounds__(128) decode_kernel(const __grid_constant__ CUt
 
   for (int k = 0;; ++k) {
     k_stop = k;
-    const int b = it.blk_begin + warp + kWarps * k;
+    const int b = it.blk_begin + (PACK ? k : warp + kWarps * k);
     if (b >= it.blk_end) break;
     const int st = k % NST;
     if (!ptx::mbar_wait(&my_bars[st], (uint32_t)((k / NST) & 1))) {
@@ -194,7 +205,7 @@ __global__ void __launch_bounds__(128) decode_kernel(const __grid_constant__ CUt
     bool bad = false;
     for (int r0 = 0; r0 < 16; r0 += box_rows) {
       const int pos = b * 16 + r0;
-      if (pos < c && pages[pos / P - first_page] < 0) bad = true;
+      if (pos < c && my_pages[pos / P - first_page] < 0) bad = true;
     }
     if (b == nblk_total - 1 || bad) {
       touched = true;
@@ -206,13 +217,13 @@ __global__ void __launch_bounds__(128) decode_kernel(const __grid_constant__ CUt
         const int r = idx / (D / 8);
         const int ch = idx % (D / 8);
         const int pos = b * 16 + r;
-        if (pos < c && pages[pos / P - first_page] >= 0) continue;
+        if (pos < c && my_pages[pos / P - first_page] >= 0) continue;
         uint4 kval = make_uint4(0, 0, 0, 0), vval = make_uint4(0, 0, 0, 0);
         if (pos == c) {
           const size_t src = ((size_t)it.token * pb.hkv + hk) * D + ch * 8;
           kval = *reinterpret_cast<const uint4 *>(kn + src);
           vval = *reinterpret_cast<const uint4 *>(vn + src);
-          const int pg = pages[c / P - first_page];
+          const int pg = my_pages[c / P - first_page];
           if (pg >= 0) {
             const size_t dst = (((size_t)pg * P + c % P) * pb.hkv + hk) * D + ch * 8;
             *reinterpret_cast<uint4 *>(kc + dst) = kval;
@@ -302,8 +313,58 @@ __global__ void __launch_bounds__(128) decode_kernel(const __grid_constant__ CUt
   // not consume, so none lands after the CTA has gone
   if (timed_out && lane == 0) {
     for (int k = k_stop; k < k_stop + NST; ++k)
-      if (it.blk_begin + warp + kWarps * k < it.blk_end)
+      if (it.blk_begin + (PACK ? k : warp + kWarps * k) < it.blk_end)
         ptx::mbar_wait(&my_bars[k % NST], (uint32_t)((k / NST) & 1));
+  }
+
+  if (PACK) {
+    // this warp's item alone: out = O / l straight from the fragments (lane
+    // holds head g0 = 8 nt + 2 (lane % 4) [+1], dims 16 mt + lane / 4 [+8])
+    if (!has_item) return;
+#pragma unroll
+    for (int nt = 0; nt < NG; ++nt) {
+      const int g0 = nt * 8 + 2 * (lane & 3);
+      // head g0 + j takes o[.][nt][j] (dim d0) and o[.][nt][j + 2] (dim d0 + 8)
+      float ov[2][KS][2];
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        ov[0][mt][0] = o[mt][nt][0];
+        ov[0][mt][1] = o[mt][nt][2];
+        ov[1][mt][0] = o[mt][nt][1];
+        ov[1][mt][1] = o[mt][nt][3];
+      }
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int g = g0 + j;
+        if (g < G) {
+          const float inv = 1.f / l_run[nt][j];
+          const float lse = (m_run[nt][j] + log2f(l_run[nt][j])) * kLn2;
+          const int h = hk * G + g;
+#pragma unroll
+          for (int mt = 0; mt < KS; ++mt) {
+            const int d0 = mt * 16 + (lane >> 2);
+            const float v0 = ov[j][mt][0] * inv, v1 = ov[j][mt][1] * inv;
+            if (it.partial < 0) {
+              __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(pb.out) + ((size_t)it.token * pb.hq + h) * D;
+              out[d0] = __float2bfloat16_rn(v0);
+              out[d0 + 8] = __float2bfloat16_rn(v1);
+            } else {
+              const size_t row = ((size_t)it.partial * pb.hkv + hk) * G + g;
+              part_o[row * D + d0] = v0;
+              part_o[row * D + d0 + 8] = v1;
+            }
+          }
+          if ((lane >> 2) == 0) {
+            if (it.partial < 0) {
+              if (pb.lse != nullptr) pb.lse[(size_t)it.token * pb.hq + h] = lse;
+            } else {
+              part_lse[((size_t)it.partial * pb.hkv + hk) * G + g] = lse;
+            }
+          }
+        }
+      }
+    }
+    return;
   }
   __syncthreads();
 
@@ -406,7 +467,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const Problem pb, const Co
   if (lane == 0 && pb.lse != nullptr) pb.lse[(size_t)ci.token * pb.hq + h] = mstar + logf(wsum);
 }
 
-template <int D, int NG>
+template <int D, int NG, bool PACK>
 cudaError_t launch_decode_t(const Problem &pb, const DecodeItem *items, int n_items, float *po, float *pl,
                             cudaStream_t stream) {
   using S = DecodeShape<D>;
@@ -417,30 +478,35 @@ cudaError_t launch_decode_t(const Problem &pb, const DecodeItem *items, int n_it
   if (!make_tmap_bf16_3d(&tk, pb.k_cache, dims, strides, box, true) ||
       !make_tmap_bf16_3d(&tv, pb.v_cache, dims, strides, box, true))
     return cudaErrorInvalidValue;
-  auto kern = decode_kernel<D, NG>;
+  auto kern = decode_kernel<D, NG, PACK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)n_items, (unsigned)pb.hkv);
-  kern<<<grid, kWarps * 32, S::kSmem, stream>>>(tk, tv, pb, items, po, pl, pb.scale * kLog2e);
+  dim3 grid((unsigned)(PACK ? (n_items + kWarps - 1) / kWarps : n_items), (unsigned)pb.hkv);
+  kern<<<grid, kWarps * 32, S::kSmem, stream>>>(tk, tv, pb, items, n_items, po, pl, pb.scale * kLog2e);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_decode(const Problem &pb, const DecodeItem *items, int n_items, float *partial_o,
-                          float *partial_lse, cudaStream_t stream) {
+                          float *partial_lse, bool pack, cudaStream_t stream) {
   if (n_items <= 0) return cudaSuccess;
   const int G = pb.hq / pb.hkv;
   const bool two = G > 8;
+#define RPA_DECODE_CASE(DD)                                                                              \
+  case DD:                                                                                               \
+    if (pack)                                                                                            \
+      return two ? launch_decode_t<DD, 2, true>(pb, items, n_items, partial_o, partial_lse, stream)      \
+                 : launch_decode_t<DD, 1, true>(pb, items, n_items, partial_o, partial_lse, stream);     \
+    return two ? launch_decode_t<DD, 2, false>(pb, items, n_items, partial_o, partial_lse, stream)       \
+               : launch_decode_t<DD, 1, false>(pb, items, n_items, partial_o, partial_lse, stream);
   switch (pb.d) {
-    case 64: return two ? launch_decode_t<64, 2>(pb, items, n_items, partial_o, partial_lse, stream)
-                        : launch_decode_t<64, 1>(pb, items, n_items, partial_o, partial_lse, stream);
-    case 128: return two ? launch_decode_t<128, 2>(pb, items, n_items, partial_o, partial_lse, stream)
-                         : launch_decode_t<128, 1>(pb, items, n_items, partial_o, partial_lse, stream);
-    case 256: return two ? launch_decode_t<256, 2>(pb, items, n_items, partial_o, partial_lse, stream)
-                         : launch_decode_t<256, 1>(pb, items, n_items, partial_o, partial_lse, stream);
+    RPA_DECODE_CASE(64)
+    RPA_DECODE_CASE(128)
+    RPA_DECODE_CASE(256)
     default: return cudaErrorInvalidValue;
   }
+#undef RPA_DECODE_CASE
 }
 
 cudaError_t launch_combine(const Problem &pb, const CombineItem *items, int n_items, const float *partial_o,

@@ -29,9 +29,10 @@ cudaError_t launch_generic(const Problem &pb, const GenericSeq *seqs,
 
 // Decode kernel (bf16): one CTA per (work item, KV head).
 // partial_o: [n_partials, Hkv, G, D] fp32; partial_lse: [n_partials, Hkv, G].
+// pack: four items per CTA, one per warp (short whole sequences).
 cudaError_t launch_decode(const Problem &pb, const DecodeItem *items,
                           int n_items, float *partial_o, float *partial_lse,
-                          cudaStream_t stream);
+                          bool pack, cudaStream_t stream);
 
 // Split-KV combine: one warp per (combine item, query head).
 cudaError_t launch_combine(const Problem &pb, const CombineItem *items,

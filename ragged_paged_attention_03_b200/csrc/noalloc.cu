@@ -176,7 +176,7 @@ extern "C" RPA_API int rpa_decode_noalloc(const void *q, const void *k_new, cons
   pb.dtype = RPA_BF16;
   pb.causal = 1;
   pb.scale = scale;
-  cudaError_t e = launch_decode(pb, d_items, ni, part_o, part_lse, stream);
+  cudaError_t e = launch_decode(pb, d_items, ni, part_o, part_lse, false, stream);
   if (e == cudaSuccess && nc > 0) e = launch_combine(pb, d_combine, nc, part_o, part_lse, stream);
   return e == cudaSuccess ? RPA_OK : RPA_ERR_CUDA;
 }

@@ -65,6 +65,7 @@ struct PrefillTile {
 struct PlanLayout {
   int64_t generic_off, n_generic_seqs, n_generic_rows;
   int64_t decode_off, n_decode_items;
+  int64_t decode_packed_off, n_decode_packed;   // short whole sequences, four per CTA
   int64_t combine_off, n_combine;
   int64_t prefill_off, n_prefill_tiles;
   int64_t n_partials;      // partial slots (per KV head) needed

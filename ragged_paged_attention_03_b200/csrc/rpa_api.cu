@@ -31,11 +31,22 @@ std::atomic<int64_t> g_opt_disable_prefill_tc{0};
 std::atomic<int64_t> g_opt_prefill_sms{0};
 std::atomic<int64_t> g_opt_concurrent_mixed{0};
 std::atomic<int64_t> g_opt_prefill_loaders{0};
+std::atomic<int64_t> g_opt_decode_pack{0};
 
 constexpr int kDefaultDecodeChunkBlocks = 192;
 // 256 blocks of 16 tokens touch at most 4096 / 8 + 1 pages, within the decode
 // kernel's 1024-entry page list.
 constexpr int kMaxDecodeChunkBlocks = 256;
+// Decode sequences this short (16-token blocks) run four per CTA, one per
+// warp; at most kMaxPackBlocks so that a warp's page-table slice (a quarter
+// of the kernel's 1024 slots) holds them at page size 8.
+constexpr int kDefaultDecodePackBlocks = 64;
+constexpr int kMaxPackBlocks = 120;
+// Packing needs enough short sequences to fill the GPU by itself (its launch
+// follows the main decode kernel): at least two packed CTAs per SM of a
+// 148-SM B200.  Fewer short sequences stay in the main kernel's item list,
+// where they fill its last wave.
+constexpr int kMinPackedCtas = 296;
 constexpr bool kHaveDecodeKernel = true;
 constexpr bool kHavePrefillKernel = true;
 
@@ -98,6 +109,7 @@ Route route_of(int32_t ql, int32_t kvl, int dtype, int cls) {
 struct HostPlan {
   std::vector<GenericSeq> generic;
   std::vector<DecodeItem> decode;
+  std::vector<DecodeItem> decode_packed;   // whole short sequences, four per CTA
   std::vector<CombineItem> combine;
   std::vector<PrefillTile> prefill;
   int32_t n_generic_rows = 0;
@@ -115,6 +127,8 @@ void build_plan(const int32_t *cu, const int32_t *kv, int32_t n, const int32_t *
   int64_t chunk = g_opt_decode_chunk.load();
   if (chunk <= 0) chunk = kDefaultDecodeChunkBlocks;
   chunk = std::min<int64_t>(chunk, kMaxDecodeChunkBlocks);
+  int64_t pack = g_opt_decode_pack.load();
+  pack = pack == 0 ? kDefaultDecodePackBlocks : std::min<int64_t>(std::max<int64_t>(pack, 0), kMaxPackBlocks);
   for (int32_t s = 0; s < n; ++s) {
     const int32_t ql = cu[s + 1] - cu[s];
     const int32_t kvl = kv[s];
@@ -140,6 +154,20 @@ void build_plan(const int32_t *cu, const int32_t *kv, int32_t n, const int32_t *
         ++hp.num_decode;
         hp.decode_bytes += (double)kvl * d->num_kv_heads * d->head_dim * 4.0;
         const int32_t nblk = (kvl + kDecodeBlock - 1) / kDecodeBlock;
+        if (nblk <= pack && nblk <= chunk) {
+          // short: the whole sequence as one item of a packed CTA
+          DecodeItem it{};
+          it.seq = s;
+          it.token = cu[s];
+          it.kv_len = kvl;
+          it.blk_begin = 0;
+          it.blk_end = nblk;
+          it.owns_new = 1;
+          it.partial = -1;
+          hp.decode_packed.push_back(it);
+          hp.decode_max_splits = std::max(hp.decode_max_splits, 1);
+          break;
+        }
         const int32_t nsplit = (int32_t)((nblk + chunk - 1) / chunk);
         const int32_t per = (nblk + nsplit - 1) / nsplit;
         hp.decode_max_splits = std::max(hp.decode_max_splits, nsplit);
@@ -190,10 +218,17 @@ void build_plan(const int32_t *cu, const int32_t *kv, int32_t n, const int32_t *
     }
   }
   // Longest decode work items first: the kernel takes items in grid order,
-  // so the short ones fill the last wave instead of trailing it.
-  std::stable_sort(hp.decode.begin(), hp.decode.end(), [](const DecodeItem &a, const DecodeItem &b) {
+  // so the short ones fill the last wave instead of trailing it (and packed
+  // CTAs get four items of similar length).
+  auto longer = [](const DecodeItem &a, const DecodeItem &b) {
     return a.blk_end - a.blk_begin > b.blk_end - b.blk_begin;
-  });
+  };
+  if ((int64_t)(hp.decode_packed.size() + 3) / 4 * d->num_kv_heads < kMinPackedCtas) {
+    hp.decode.insert(hp.decode.end(), hp.decode_packed.begin(), hp.decode_packed.end());
+    hp.decode_packed.clear();
+  }
+  std::stable_sort(hp.decode.begin(), hp.decode.end(), longer);
+  std::stable_sort(hp.decode_packed.begin(), hp.decode_packed.end(), longer);
   // Heaviest prefill tiles first: with a causal mask a tile's key range ends
   // at its last row, so later tiles of a sequence carry more work.
   std::stable_sort(hp.prefill.begin(), hp.prefill.end(),
@@ -211,6 +246,9 @@ void build_plan(const int32_t *cu, const int32_t *kv, int32_t n, const int32_t *
   L.decode_off = off;
   L.n_decode_items = (int64_t)hp.decode.size();
   off += L.n_decode_items * (int64_t)(sizeof(DecodeItem) / 4);
+  L.decode_packed_off = off;
+  L.n_decode_packed = (int64_t)hp.decode_packed.size();
+  off += L.n_decode_packed * (int64_t)(sizeof(DecodeItem) / 4);
   L.combine_off = off;
   L.n_combine = (int64_t)hp.combine.size();
   off += L.n_combine * (int64_t)(sizeof(CombineItem) / 4);
@@ -227,6 +265,8 @@ void serialize(const HostPlan &hp, int32_t *dst) {
     memcpy(dst + L.generic_off, hp.generic.data(), hp.generic.size() * sizeof(GenericSeq));
   if (!hp.decode.empty())
     memcpy(dst + L.decode_off, hp.decode.data(), hp.decode.size() * sizeof(DecodeItem));
+  if (!hp.decode_packed.empty())
+    memcpy(dst + L.decode_packed_off, hp.decode_packed.data(), hp.decode_packed.size() * sizeof(DecodeItem));
   if (!hp.combine.empty())
     memcpy(dst + L.combine_off, hp.combine.data(), hp.combine.size() * sizeof(CombineItem));
   if (!hp.prefill.empty())
@@ -388,6 +428,7 @@ extern "C" RPA_API int64_t rpa_set_option(int32_t option, int64_t value) {
     case RPA_OPT_PREFILL_SMS: return g_opt_prefill_sms.exchange(value);
     case RPA_OPT_CONCURRENT_MIXED: return g_opt_concurrent_mixed.exchange(value);
     case RPA_OPT_PREFILL_LOADERS: return g_opt_prefill_loaders.exchange(value);
+    case RPA_OPT_DECODE_PACK_BLOCKS: return g_opt_decode_pack.exchange(value);
     default: return -1;
   }
 }
@@ -403,7 +444,8 @@ extern "C" RPA_API int rpa_plan(const int32_t *cu_q_lens, const int32_t *kv_lens
     info->num_prefill = hp.num_prefill;
     info->num_generic = hp.num_generic;
     info->num_empty = hp.num_empty;
-    info->decode_items = (int32_t)hp.decode.size();
+    info->decode_items = (int32_t)(hp.decode.size() + hp.decode_packed.size());
+    info->decode_packed = (int32_t)hp.decode_packed.size();
     info->decode_max_splits = hp.decode_max_splits;
     info->combine_rows = (int32_t)hp.combine.size();
     info->prefill_tiles = (int32_t)hp.prefill.size();
@@ -479,7 +521,8 @@ extern "C" RPA_API int rpa_forward(const void *q, const void *k_new, const void 
     // concurrently: the compute-bound prefill kernel on the side stream with a
     // share of the SMs, the bandwidth-bound decode kernel on the caller's
     // stream on the rest.
-    const bool mixed = L.n_prefill_tiles > 0 && (L.n_decode_items > 0 || L.n_generic_rows > 0) &&
+    const bool mixed = L.n_prefill_tiles > 0 &&
+                       (L.n_decode_items > 0 || L.n_decode_packed > 0 || L.n_generic_rows > 0) &&
                        g_opt_concurrent_mixed.load() != 0;
     cudaStream_t pstream = stream;
     int prefill_ctas = 0;
@@ -511,7 +554,12 @@ extern "C" RPA_API int rpa_forward(const void *q, const void *k_new, const void 
     if (L.n_decode_items > 0 && e == cudaSuccess)
       e = traced(RPA_KERNEL_DECODE, stream, [&] {
         return launch_decode(pb, (const DecodeItem *)(slot.dev + L.decode_off),
-                             (int)L.n_decode_items, partial_o, partial_lse, stream);
+                             (int)L.n_decode_items, partial_o, partial_lse, false, stream);
+      });
+    if (L.n_decode_packed > 0 && e == cudaSuccess)
+      e = traced(RPA_KERNEL_DECODE, stream, [&] {
+        return launch_decode(pb, (const DecodeItem *)(slot.dev + L.decode_packed_off),
+                             (int)L.n_decode_packed, partial_o, partial_lse, true, stream);
       });
     if (L.n_combine > 0 && e == cudaSuccess)
       e = traced(RPA_KERNEL_COMBINE, stream, [&] {

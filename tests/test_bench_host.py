@@ -98,12 +98,12 @@ def test_roofline_uses_the_dominant_kernel():
             "prefill_flops": 10 ** 12}
     pk = {"hbm": 8000.0, "tc": 2000.0, "tc_sustained": 1500.0, "source": "test"}
     # decode dominates: 2 launches of 0.25 ms each move 2 GB per launch
-    r = bench.roofline("decode_128", work, {"decode": (2, 0.5), "combine": (2, 0.05)}, pk)
+    r = bench.roofline("decode_128", work, {"decode": (2, 0.5), "combine": (2, 0.05)}, pk, 2)
     assert r["kernel"] == "decode" and r["bound"] == "hbm"
     assert r["achieved"] == pytest.approx(2e9 / 0.25e-3 / 1e9)
     assert r["frac"] == pytest.approx(r["achieved"] / 8000.0)
     # prefill dominates: 1 launch of 1 ms does 1 TFLOP
-    r = bench.roofline("mixed_96d_4c", work, {"decode": (1, 0.2), "prefill": (1, 1.0)}, pk)
+    r = bench.roofline("mixed_96d_4c", work, {"decode": (1, 0.2), "prefill": (1, 1.0)}, pk, 1)
     assert r["kernel"] == "prefill" and r["bound"] == "tensor"
     assert r["achieved"] == pytest.approx(1000.0)
     assert r["kernel_share"]["prefill"] == pytest.approx(1.0 / 1.2, abs=1e-4)

@@ -127,6 +127,32 @@ def test_decode_chunking(rb):
         pytest.skip("decode kernel not routed")
     assert info.decode_items == 1 + 2 + 1
     assert info.combine_rows == 1 and info.decode_max_splits == 2
+    # three sequences are too few to pack (they would not fill the GPU)
+    assert info.decode_packed == 0
+
+
+def test_decode_packing(rb):
+    """Whole sequences of at most RPA_OPT_DECODE_PACK_BLOCKS blocks (default
+    64) run four per CTA, one per warp, when there are enough of them to
+    fill 296 CTAs (two per SM); < 0 turns packing off."""
+    # 150 of each: 1, 64, 65 and 119 blocks; 8 KV heads -> 38 * 8 = 304 packed CTAs
+    kv = [5] * 150 + [16 * 64] * 150 + [16 * 64 + 1] * 150 + [1900] * 150
+    info = plan(rb, [1] * len(kv), kv, max_pages_per_seq=128)
+    if info.num_decode == 0:
+        pytest.skip("decode kernel not routed")
+    assert info.decode_packed == 300 and info.decode_items == 600
+    # too few short sequences: they stay in the main decode launch
+    info = plan(rb, [1] * 4, [5, 16 * 64, 16 * 64 + 1, 1900], max_pages_per_seq=128)
+    assert info.decode_packed == 0 and info.decode_items == 4
+    old = rb.rpa_set_option(rb.RPA_OPT_DECODE_PACK_BLOCKS, -1)
+    try:
+        info = plan(rb, [1] * len(kv), kv, max_pages_per_seq=128)
+        assert info.decode_packed == 0 and info.decode_items == 600
+        rb.rpa_set_option(rb.RPA_OPT_DECODE_PACK_BLOCKS, 1000)     # clamped to 120 blocks
+        info = plan(rb, [1] * len(kv), kv, max_pages_per_seq=128)
+        assert info.decode_packed == 600
+    finally:
+        rb.rpa_set_option(rb.RPA_OPT_DECODE_PACK_BLOCKS, old)
 
 
 def test_workload_plans(rb):

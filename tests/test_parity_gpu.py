@@ -174,6 +174,33 @@ def test_more_shapes(oracle_mod, case, loaders):
         binding.rpa_set_option(binding.RPA_OPT_PREFILL_LOADERS, old)
 
 
+@pytest.mark.parametrize("pack", [0, -1])
+@pytest.mark.parametrize("shape", [(16, 1, 64, 8), (32, 8, 128, 16), (64, 4, 256, 64)])
+def test_packed_short_decode(oracle_mod, pack, shape):
+    """Short decode sequences run four per CTA (one per warp; the last CTA
+    holds one), against the same batch with packing off."""
+    from ragged_paged_attention_03_b200 import binding
+    hq, hkv, d, p = shape
+    old = binding.rpa_set_option(binding.RPA_OPT_DECODE_PACK_BLOCKS, pack)
+    try:
+        # enough short sequences to be packed (>= 296 packed CTAs); the last CTA holds one
+        base = [1, 2, 15, 16, 17, 31, 100, 200, 255, 256, 257, 400, 511]
+        n = 4 * (296 // hkv + 1) + 1
+        kv = [base[i % len(base)] for i in range(n)]
+        prob = I.make_problem([1] * len(kv), kv, num_q_heads=hq, num_kv_heads=hkv, head_dim=d,
+                              page_size=p, dtype=I.BF16, seed=700 + d, pool=1.5)
+        if pack == 0:
+            from ragged_paged_attention_03_b200 import binding as rb
+            info = rb.rpa_plan(prob.cu_q_lens, prob.kv_lens, None,
+                               rb.rpa_dims(num_q_heads=hq, num_kv_heads=hkv, head_dim=d, page_size=p,
+                                           num_pages=prob.num_pages, max_pages_per_seq=prob.page_table.shape[1],
+                                           total_q_tokens=len(kv), dtype=I.BF16))
+            assert info.decode_packed == len(kv)
+        full_check(oracle_mod, prob)
+    finally:
+        binding.rpa_set_option(binding.RPA_OPT_DECODE_PACK_BLOCKS, old)
+
+
 def test_bad_page_is_flagged_not_read(oracle_mod):
     """A page-table entry outside the pool is reported through the device
     error word; the kernels never dereference it."""
