@@ -53,8 +53,11 @@ enum {
   RPA_ERR_DISTRIBUTION = 4,  /* distribution given and inconsistent */
   RPA_ERR_OOM = 5,           /* library workspace could not be allocated */
   RPA_ERR_CUDA = 6,          /* a CUDA call or kernel launch failed */
-  RPA_ERR_SCRATCH_LIMIT = 7  /* rpa_decode_noalloc: the batch needs more
+  RPA_ERR_SCRATCH_LIMIT = 7, /* rpa_decode_noalloc: the batch needs more
                                 scratch than its fixed array holds */
+  RPA_ERR_WORKSPACE = 8      /* rpa_forward_device: the caller's workspace
+                                is smaller than rpa_device_workspace_size
+                                reports or not 256-byte aligned */
 };
 
 /* Bits of the device error word read by rpa_device_status(). */
@@ -64,6 +67,12 @@ enum {
 #define RPA_DEV_TIMEOUT 0x2u  /* a bounded wait on a shared-memory barrier ran
                                  out; the CTA stopped early, outputs of that
                                  CTA are incomplete */
+#define RPA_DEV_BAD_LENGTHS 0x4u /* rpa_forward_device: the device-resident
+                                 lengths broke a rule rpa_forward checks on the
+                                 host (RPA_ERR_LENGTHS) or num_seqs was
+                                 outside [0, max_seqs]; the call did nothing
+                                 else: no cache slot, out or lse row was
+                                 written */
 
 /* Problem geometry. */
 typedef struct {
@@ -261,6 +270,65 @@ RPA_API int rpa_decode_noalloc(const void *q, const void *k_new,
                                float scale, void *out, float *lse,
                                const rpa_dims *dims, uint32_t *dev_flags,
                                void *stream);
+
+/*
+ * rpa_device_workspace_size -- bytes of device workspace rpa_forward_device
+ * needs for batches of at most max_seqs sequences under dims (total_q_tokens
+ * is the row capacity T of q / k_new / v_new / out).  It depends on dims,
+ * max_seqs and the current RPA_OPT_DECODE_CHUNK_BLOCKS and
+ * RPA_OPT_DECODE_PACK_BLOCKS values only.  Host only; returns RPA_OK or the
+ * RPA_ERR_* code of bad dims / max_seqs < 0 (then *bytes = 0).
+ */
+RPA_API int rpa_device_workspace_size(const rpa_dims *dims, int32_t max_seqs,
+                                      int64_t *bytes);
+
+/*
+ * rpa_forward_device -- rpa_forward with the metadata pass on the GPU, for
+ * CUDA-graph capture.  The pages propose moving the kernel's scalar metadata
+ * work off the main compute path (arXiv 2604.15464, future work: SparseCore
+ * offload); here a one-CTA planner kernel, queued on `stream` before the
+ * attention kernels, reads the lengths from device memory and writes the
+ * work lists into `workspace`.
+ *
+ * Differences from rpa_forward:
+ *   cu_q_lens [max_seqs + 1], kv_lens [max_seqs] and num_seqs [1] are DEVICE
+ *     int32 arrays, read by the planner kernel when it runs, so the caller may
+ *     rewrite them (and q / k_new / v_new) between replays of a captured
+ *     graph.  Entries past num_seqs are not read.
+ *   dims->total_q_tokens is a capacity T: q, k_new, v_new, out (and lse)
+ *     have T rows, cu_q_lens[num_seqs] <= T, and rows from cu_q_lens[num_seqs]
+ *     on are not written.  page_table has max_seqs rows.
+ *   No distribution: sequences are routed by q_len (1: decode kernel, > 1:
+ *     prefill kernel, 0: nothing); fp32 I/O runs on the generic kernel.
+ *   workspace: caller-owned device memory, 256-byte aligned, of at least
+ *     rpa_device_workspace_size(dims, max_seqs) bytes (measured with the same
+ *     option values), else RPA_ERR_WORKSPACE.  Calls that share a workspace
+ *     must be ordered on the device.  The library allocates nothing.
+ *   dev_flags: device uint32 that receives RPA_DEV_* bits (OR-ed in, never
+ *     cleared), or NULL to drop them.  Lengths that rpa_forward would reject
+ *     with RPA_ERR_LENGTHS set RPA_DEV_BAD_LENGTHS and the call writes
+ *     nothing.
+ *   The kernels launched, their grids (sized for the workspace's capacity)
+ *     and arguments depend only on the pointers, dims, max_seqs, scale,
+ *     causal and the option values, never on the lengths: the host neither
+ *     reads device memory nor waits, so the call can be captured into a CUDA
+ *     graph and replayed.  The head_dim <= 128 prefill kernel takes one TMA
+ *     producer warp for K and V unless RPA_OPT_PREFILL_LOADERS is 2.
+ * Results (out, lse, cache contents) are those rpa_forward gives for the same
+ * batch.  max_seqs == 0 or T == 0 is a successful no-op.  Host-side checks
+ * (scale, dims, null pointers, workspace) return RPA_ERR_* before anything is
+ * queued; RPA_ERR_CUDA if a launch failed.
+ */
+RPA_API int rpa_forward_device(const void *q, const void *k_new,
+                               const void *v_new, void *k_cache,
+                               void *v_cache, const int32_t *page_table,
+                               const int32_t *cu_q_lens,
+                               const int32_t *kv_lens,
+                               const int32_t *num_seqs, int32_t max_seqs,
+                               float scale, int32_t causal, void *out,
+                               float *lse, const rpa_dims *dims,
+                               void *workspace, int64_t workspace_bytes,
+                               uint32_t *dev_flags, void *stream);
 
 #ifdef __cplusplus
 }

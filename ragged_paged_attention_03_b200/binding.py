@@ -77,6 +77,13 @@ _lib.rpa_decode_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _P, _i32, ctypes.c_f
                                     ctypes.POINTER(rpa_dims), _P, _P]
 _lib.rpa_decode_noalloc.restype = ctypes.c_int
 RPA_ERR_SCRATCH_LIMIT = 7
+RPA_ERR_WORKSPACE = 8
+RPA_DEV_BAD_LENGTHS = 0x4
+_lib.rpa_device_workspace_size.argtypes = [ctypes.POINTER(rpa_dims), _i32, ctypes.POINTER(ctypes.c_int64)]
+_lib.rpa_device_workspace_size.restype = ctypes.c_int
+_lib.rpa_forward_device.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _i32, ctypes.c_float, _i32, _P, _P,
+                                    ctypes.POINTER(rpa_dims), _P, ctypes.c_int64, _P, _P]
+_lib.rpa_forward_device.restype = ctypes.c_int
 
 
 def library() -> ctypes.CDLL:
@@ -210,3 +217,48 @@ def rpa_decode_noalloc(q, k_new, v_new, k_cache, v_cache, page_table, kv_lens, s
                                  ctypes.byref(dims), _dev(dev_flags, "dev_flags", torch.int32), sptr)
     if rc != RPA_OK:
         raise RpaError(rc, "rpa_decode_noalloc")
+
+
+def rpa_device_workspace_size(dims: rpa_dims, max_seqs: int) -> int:
+    """Bytes of device workspace rpa_forward_device needs for these dims and
+    at most `max_seqs` sequences."""
+    n = ctypes.c_int64(0)
+    rc = _lib.rpa_device_workspace_size(ctypes.byref(dims), int(max_seqs), ctypes.byref(n))
+    if rc != RPA_OK:
+        raise RpaError(rc, "rpa_device_workspace_size")
+    return int(n.value)
+
+
+def rpa_forward_device(q, k_new, v_new, k_cache, v_cache, page_table, cu_q_lens, kv_lens, num_seqs,
+                       scale: float, causal: bool, out, workspace, lse=None, dev_flags=None,
+                       stream=None) -> None:
+    """Calls rpa_forward_device: the lengths stay on the device and the
+    planning runs in a kernel, so the call can be captured in a CUDA graph.
+
+    cu_q_lens [max_seqs+1], kv_lens [max_seqs], num_seqs [1]: int32 CUDA
+    tensors (max_seqs = kv_lens.numel()); page_table has max_seqs rows; q's
+    row count is the token capacity T.  workspace: uint8 CUDA tensor of at
+    least rpa_device_workspace_size bytes.  dev_flags: optional int32 CUDA
+    tensor of one element that receives the device error bits."""
+    dt = q.dtype
+    for name, t in (("k_new", k_new), ("v_new", v_new), ("k_cache", k_cache),
+                    ("v_cache", v_cache), ("out", out)):
+        if t.dtype != dt:
+            raise TypeError(f"{name} dtype {t.dtype} != q dtype {dt}")
+    max_seqs = kv_lens.numel()
+    if cu_q_lens.numel() < max_seqs + 1 or num_seqs.numel() < 1 or page_table.shape[0] < max_seqs:
+        raise ValueError("cu_q_lens needs max_seqs + 1 entries, num_seqs one, page_table max_seqs rows")
+    dims = make_dims(q, k_cache, page_table)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    sptr = ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+    rc = _lib.rpa_forward_device(_dev(q, "q"), _dev(k_new, "k_new"), _dev(v_new, "v_new"),
+                                 _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                                 _dev(page_table, "page_table", torch.int32),
+                                 _dev(cu_q_lens, "cu_q_lens", torch.int32), _dev(kv_lens, "kv_lens", torch.int32),
+                                 _dev(num_seqs, "num_seqs", torch.int32), max_seqs, float(scale),
+                                 int(bool(causal)), _dev(out, "out"), _dev(lse, "lse", torch.float32),
+                                 ctypes.byref(dims), _dev(workspace, "workspace", torch.uint8),
+                                 workspace.numel(), _dev(dev_flags, "dev_flags", torch.int32), sptr)
+    if rc != RPA_OK:
+        raise RpaError(rc, "rpa_forward_device")

@@ -77,6 +77,9 @@ __global__ void __launch_bounds__(128) decode_kernel(const __grid_constant__ CUt
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  if (pb.dev_counts != nullptr) n_items = min(n_items, pb.dev_counts[PACK ? kCntPacked : kCntDecode]);
+  // capacity-sized grid of a device-planned call: CTAs past the work leave
+  if ((PACK ? (int)blockIdx.x * kWarps : (int)blockIdx.x) >= n_items) return;
   const int item_idx = PACK ? (int)blockIdx.x * kWarps + warp : (int)blockIdx.x;
   const bool has_item = item_idx < n_items;   // PACK: the last CTA may hold fewer items
   DecodeItem it = items[has_item ? item_idx : 0];
@@ -432,6 +435,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const Problem pb, const Co
   constexpr int E = D / 32;
   const int lane = threadIdx.x & 31;
   const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (pb.dev_counts != nullptr) n_items = min(n_items, pb.dev_counts[kCntCombine]);
   if (w >= (long long)n_items * pb.hq) return;
   const CombineItem ci = items[w / pb.hq];
   const int h = (int)(w % pb.hq);

@@ -33,6 +33,10 @@ __global__ void __launch_bounds__(128) generic_kernel(Problem pb, const GenericS
   constexpr int E = D / 32;  // elements per lane
   const int lane = threadIdx.x & 31;
   const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (pb.dev_counts != nullptr) {
+    n_seqs = min(n_seqs, pb.dev_counts[kCntGenericSeqs]);
+    n_rows = min(n_rows, pb.dev_counts[kCntGenericRows]);
+  }
   if (warp >= (long long)n_rows * pb.hq) return;
   const int row = (int)(warp / pb.hq);
   const int h = (int)(warp % pb.hq);

@@ -1,0 +1,29 @@
+// host_common.h -- host-side helpers shared by the entry points of the
+// library (rpa_api.cu, device_plan.cu): geometry validation and the
+// effective values of the process-wide planner options.
+#pragma once
+#include <stdint.h>
+
+#include "rpa.h"
+
+namespace rpa {
+
+// RPA_OK, or the RPA_ERR_* code rpa_forward returns for these dims.
+int validate_dims(const rpa_dims *d);
+
+// Effective planner options (defaults and clamps applied).
+int64_t decode_chunk_blocks();   // 16-token blocks per decode work item
+int64_t decode_pack_blocks();    // longest packed decode sequence, 0 = never
+int64_t prefill_loaders();       // RPA_OPT_PREFILL_LOADERS as set (0, 1, 2)
+
+// Packed decode CTAs a batch must fill before packing is used (two per SM
+// of a 148-SM B200): a packed launch follows the main decode launch, so a
+// few short sequences are better placed in that launch's last wave.
+constexpr int kMinPackedCtas = 296;
+
+// Largest decode work item, in 16-token blocks: 256 blocks of 16 tokens
+// touch at most 4096 / 8 + 1 pages, within the decode kernel's 1024-entry
+// page list.
+constexpr int kMaxDecodeChunkBlocks = 256;
+
+}  // namespace rpa

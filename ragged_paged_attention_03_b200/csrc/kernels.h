@@ -21,6 +21,10 @@ struct Problem {
   int32_t hq, hkv, d, p, num_pages, max_pages, dtype, causal;
   int32_t total_q;     // T: rows of q, k_new, v_new, out
   float scale;
+  // Device-planned calls: the work counts (DeviceCount slots) written by the
+  // planner kernel; each kernel takes min(its slot, the count it was launched
+  // for).  nullptr: the launch counts are exact (host plan).
+  const int32_t *dev_counts;
 };
 
 // Generic SIMT kernel: any dtype, any q_len, one warp per (row, query head).

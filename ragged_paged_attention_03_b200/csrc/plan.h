@@ -61,6 +61,21 @@ struct PrefillTile {
   int32_t pad;
 };
 
+// Device-planned calls (rpa_forward_device): the planner kernel writes the
+// work counts into a header of int32 slots; each kernel of the call is
+// launched with a grid sized for the workspace's capacity and bounds its work
+// by its slot.  Host-planned calls pass no header.
+enum DeviceCount {
+  kCntDecode = 0,       // decode work items
+  kCntPacked = 1,       // packed (four per CTA) decode items
+  kCntCombine = 2,      // combine rows
+  kCntPrefill = 3,      // prefill tiles
+  kCntGenericSeqs = 4,  // generic-kernel sequences
+  kCntGenericRows = 5,  // generic-kernel rows
+  kCntPartials = 6,     // split-KV partial slots in use
+  kCntSlots = 8
+};
+
 // Offsets (in int32 units) of each section inside the plan blob.
 struct PlanLayout {
   int64_t generic_off, n_generic_seqs, n_generic_rows;

@@ -572,7 +572,10 @@ __device__ __forceinline__ void cache_update(const Problem pb, const PrefillTile
 // Every barrier parity runs on counters that span units, so the producer
 // loads the next unit's Q and K/V while the current one finishes and the MMA
 // warp starts the next unit while the softmax warps are still storing O.
-template <int D, bool SPLIT>
+// DEV: a device-planned call (capacity-sized grid, the unit count read from
+// pb.dev_counts); a separate instance so that the host-planned build keeps
+// its count in the kernel parameters rather than in a register.
+template <int D, bool SPLIT, bool DEV>
 __global__ void __launch_bounds__(384, 1)
     prefill2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
                     const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_kn,
@@ -592,6 +595,11 @@ __global__ void __launch_bounds__(384, 1)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  if (DEV) {
+    // capacity-sized grid: CTAs without a unit leave before any set-up
+    n_units = min(n_units, pb.dev_counts[kCntPrefill] * pb.hq);
+    if ((int)blockIdx.x >= n_units) return;
+  }
 
   if (tid == 0) {
     ptx::mbar_init(&bars->q_full, 1);
@@ -822,7 +830,9 @@ cudaError_t launch_t(const Problem &pb, const PrefillTile *tiles, int n_tiles, i
       !make_tmap_bf16_3d(&tkn, pb.k_new, ndims, nstr, nbox, true) ||
       !make_tmap_bf16_3d(&tvn, pb.v_new, ndims, nstr, nbox, true))
     return cudaErrorInvalidValue;
-  auto kern = split ? prefill2_kernel<D, true> : prefill2_kernel<D, false>;
+  const bool dev = pb.dev_counts != nullptr;
+  auto kern = split ? (dev ? prefill2_kernel<D, true, true> : prefill2_kernel<D, true, false>)
+                    : (dev ? prefill2_kernel<D, false, true> : prefill2_kernel<D, false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem);
   if (e != cudaSuccess) return e;
   const int n_units = n_tiles * pb.hq;

@@ -113,6 +113,8 @@ __global__ void __launch_bounds__(192, 1)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  // capacity-sized grid of a device-planned call: CTAs past the tiles leave
+  if (pb.dev_counts != nullptr && (int)blockIdx.y >= pb.dev_counts[kCntPrefill]) return;
   const PrefillTile tile = tiles[blockIdx.y];
   const int h = blockIdx.x;
   const int G = pb.hq / pb.hkv;

@@ -18,6 +18,7 @@
 #include <new>
 #include <vector>
 
+#include "host_common.h"
 #include "kernels.h"
 #include "plan.h"
 #include "rpa.h"
@@ -34,23 +35,30 @@ std::atomic<int64_t> g_opt_prefill_loaders{0};
 std::atomic<int64_t> g_opt_decode_pack{0};
 
 constexpr int kDefaultDecodeChunkBlocks = 192;
-// 256 blocks of 16 tokens touch at most 4096 / 8 + 1 pages, within the decode
-// kernel's 1024-entry page list.
-constexpr int kMaxDecodeChunkBlocks = 256;
 // Decode sequences this short (16-token blocks) run four per CTA, one per
 // warp; at most kMaxPackBlocks so that a warp's page-table slice (a quarter
 // of the kernel's 1024 slots) holds them at page size 8.
 constexpr int kDefaultDecodePackBlocks = 64;
 constexpr int kMaxPackBlocks = 120;
-// Packing needs enough short sequences to fill the GPU by itself (its launch
-// follows the main decode kernel): at least two packed CTAs per SM of a
-// 148-SM B200.  Fewer short sequences stay in the main kernel's item list,
-// where they fill its last wave.
-constexpr int kMinPackedCtas = 296;
 constexpr bool kHaveDecodeKernel = true;
 constexpr bool kHavePrefillKernel = true;
 
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+}  // namespace
+
+int64_t decode_chunk_blocks() {
+  int64_t chunk = g_opt_decode_chunk.load();
+  if (chunk <= 0) chunk = kDefaultDecodeChunkBlocks;
+  return std::min<int64_t>(chunk, kMaxDecodeChunkBlocks);
+}
+
+int64_t decode_pack_blocks() {
+  const int64_t pack = g_opt_decode_pack.load();
+  return pack == 0 ? kDefaultDecodePackBlocks : std::min<int64_t>(std::max<int64_t>(pack, 0), kMaxPackBlocks);
+}
+
+int64_t prefill_loaders() { return g_opt_prefill_loaders.load(); }
 
 int validate_dims(const rpa_dims *d) {
   if (d == nullptr) return RPA_ERR_INVALID_ARG;
@@ -64,6 +72,8 @@ int validate_dims(const rpa_dims *d) {
   if (d->num_q_heads / d->num_kv_heads > 16) return RPA_ERR_UNSUPPORTED;
   return RPA_OK;
 }
+
+namespace {
 
 int validate_lengths(const int32_t *cu, const int32_t *kv, int32_t n, const rpa_dims *d) {
   if (n < 0) return RPA_ERR_INVALID_ARG;
@@ -124,11 +134,8 @@ struct HostPlan {
 
 void build_plan(const int32_t *cu, const int32_t *kv, int32_t n, const int32_t *dist,
                 const rpa_dims *d, HostPlan &hp) {
-  int64_t chunk = g_opt_decode_chunk.load();
-  if (chunk <= 0) chunk = kDefaultDecodeChunkBlocks;
-  chunk = std::min<int64_t>(chunk, kMaxDecodeChunkBlocks);
-  int64_t pack = g_opt_decode_pack.load();
-  pack = pack == 0 ? kDefaultDecodePackBlocks : std::min<int64_t>(std::max<int64_t>(pack, 0), kMaxPackBlocks);
+  const int64_t chunk = decode_chunk_blocks();
+  const int64_t pack = decode_pack_blocks();
   for (int32_t s = 0; s < n; ++s) {
     const int32_t ql = cu[s + 1] - cu[s];
     const int32_t kvl = kv[s];
@@ -416,6 +423,7 @@ extern "C" RPA_API const char *rpa_status_string(int status) {
     case RPA_ERR_OOM: return "workspace allocation failed";
     case RPA_ERR_CUDA: return "CUDA error";
     case RPA_ERR_SCRATCH_LIMIT: return "batch exceeds the no-alloc scratch limit";
+    case RPA_ERR_WORKSPACE: return "workspace too small or misaligned";
     default: return "unknown status";
   }
 }

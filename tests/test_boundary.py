@@ -213,3 +213,52 @@ def test_forward_rejects_non_positive_scale(rb, scale):
     rc = lib.rpa_decode_noalloc(fake, fake, fake, fake, fake, fake, kv.ctypes.data_as(ctypes.c_void_p), 1,
                                 ctypes.c_float(scale), fake, None, ctypes.byref(d), None, None)
     assert rc == 1
+
+
+def test_device_workspace_size(rb):
+    """The device-planned call's workspace depends on the geometry, the
+    sequence capacity and the decode options only, and grows with each."""
+    d = dims(total_q_tokens=128, max_pages_per_seq=512)
+    assert rb.rpa_device_workspace_size(d, 0) == 256            # the header alone
+    sizes = [rb.rpa_device_workspace_size(d, n) for n in (1, 16, 128)]
+    assert sizes[0] < sizes[1] < sizes[2]
+    assert all(s % 256 == 0 for s in sizes)
+    # longer contexts allow more split-KV chunks, hence more partial slots
+    assert rb.rpa_device_workspace_size(dims(total_q_tokens=128, max_pages_per_seq=2048), 128) > sizes[2]
+    # fp32 runs on the generic kernel: no decode items, no partials
+    assert rb.rpa_device_workspace_size(dims(total_q_tokens=128, max_pages_per_seq=512, dtype=0), 128) < sizes[2]
+    old = rb.rpa_set_option(rb.RPA_OPT_DECODE_CHUNK_BLOCKS, 16)
+    try:
+        assert rb.rpa_device_workspace_size(d, 128) > sizes[2]
+    finally:
+        rb.rpa_set_option(rb.RPA_OPT_DECODE_CHUNK_BLOCKS, old)
+    with pytest.raises(rb.RpaError) as e:
+        rb.rpa_device_workspace_size(d, -1)
+    assert e.value.code == 1
+    with pytest.raises(rb.RpaError) as e:
+        rb.rpa_device_workspace_size(dims(head_dim=96), 4)
+    assert e.value.code == 2
+
+
+def test_forward_device_host_checks(rb):
+    """rpa_forward_device rejects bad scale, pointers and workspaces on the
+    host, before anything is queued; an empty capacity is a no-op."""
+    lib = rb.library()
+    d = dims(total_q_tokens=8)
+    need = rb.rpa_device_workspace_size(d, 4)
+    fake = ctypes.c_void_p(0x10000)
+
+    def call(ws=fake, ws_bytes=need, scale=1.0, max_seqs=4, cu=fake, dd=d):
+        return lib.rpa_forward_device(fake, fake, fake, fake, fake, fake, cu, fake, fake, max_seqs,
+                                      ctypes.c_float(scale), 1, fake, None, ctypes.byref(dd), ws, ws_bytes,
+                                      None, None)
+    assert call(ws_bytes=need - 1) == rb.RPA_ERR_WORKSPACE
+    assert call(ws=ctypes.c_void_p(0x10000 + 64)) == rb.RPA_ERR_WORKSPACE    # not 256-byte aligned
+    assert call(ws=None) == 1
+    assert call(cu=None) == 1
+    assert call(scale=0.0) == 1
+    assert call(max_seqs=-1) == 1
+    assert call(dd=dims(head_dim=96, total_q_tokens=8)) == 2
+    assert call(max_seqs=0) == 0                  # no sequence slot: nothing to do
+    assert call(dd=dims(total_q_tokens=0)) == 0   # no token row: nothing to do
+    assert rb.rpa_status_string(rb.RPA_ERR_WORKSPACE) == "workspace too small or misaligned"
