@@ -204,6 +204,72 @@ def time_steps(prob, steps, warmup, flush, stream, profile=False):
     return ms, kern
 
 
+def time_graph(prob, steps, warmup, flush, stream):
+    """rpa_forward_device (lengths in device memory, planned by a kernel)
+    captured once in a CUDA graph and replayed every step.  Returns the mean
+    device ms per step and the host microseconds one replay takes to launch."""
+    from ragged_paged_attention_03_b200 import binding
+    dev = prob.q.device
+    out = torch.empty_like(prob.q)
+    lse = torch.empty(prob.q.shape[0], prob.num_q_heads, dtype=torch.float32, device=dev)
+    cu = torch.as_tensor(np.asarray(prob.cu_q_lens), dtype=torch.int32).to(dev)
+    kv = torch.as_tensor(np.asarray(prob.kv_lens), dtype=torch.int32).to(dev)
+    n = torch.tensor([prob.num_seqs], dtype=torch.int32, device=dev)
+    flags = torch.zeros(1, dtype=torch.int32, device=dev)
+    dims = binding.make_dims(prob.q, prob.k_cache, prob.page_table)
+    ws = torch.empty(binding.rpa_device_workspace_size(dims, prob.num_seqs), dtype=torch.uint8, device=dev)
+
+    def call():
+        binding.rpa_forward_device(prob.q, prob.k_new, prob.v_new, prob.k_cache, prob.v_cache,
+                                   prob.page_table, cu, kv, n, prob.scale, prob.causal, out, ws,
+                                   lse=lse, dev_flags=flags)
+
+    with torch.cuda.stream(stream):
+        call()
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            call()
+        for _ in range(warmup):
+            flush.add_(1)
+            graph.replay()
+        stream.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        host = []
+        for a, b in evs:
+            flush.add_(1)
+            a.record(stream)
+            t0 = time.perf_counter()
+            graph.replay()
+            host.append(time.perf_counter() - t0)
+            b.record(stream)
+        stream.synchronize()
+    if int(flags.item()):
+        raise RuntimeError(f"device error flags {int(flags.item()):#x}")
+    del graph
+    ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    return ms, float(np.median(host)) * 1e6
+
+
+def host_call_us(prob, calls, stream):
+    """Host microseconds one host-planned rpa_forward call takes (planning,
+    plan upload and launches), median over `calls`."""
+    from ragged_paged_attention_03_b200 import binding
+    out = torch.empty_like(prob.q)
+    lse = torch.empty(prob.q.shape[0], prob.num_q_heads, dtype=torch.float32, device=prob.q.device)
+    ts = []
+    with torch.cuda.stream(stream):
+        for _ in range(calls):
+            t0 = time.perf_counter()
+            binding.rpa_forward(prob.q, prob.k_new, prob.v_new, prob.k_cache, prob.v_cache,
+                                prob.page_table, prob.cu_q_lens, prob.kv_lens, prob.distribution,
+                                prob.scale, prob.causal, out, lse, stream=stream)
+            ts.append(time.perf_counter() - t0)
+            stream.synchronize()
+    return float(np.median(ts)) * 1e6
+
+
 def time_e2e(prob, steps, warmup, flush, stream):
     """Host buffers in, host buffers out: each step copies this step's Q, new
     K/V and page table from pinned host memory, runs rpa_forward and copies
@@ -436,6 +502,9 @@ def main():
             torch.distributed.barrier()
         e2e_ms, h2d, d2h = time_e2e(prob, max(10, args.steps // 4), 3, flush, stream)
         e2e_ms = max_over_ranks(e2e_ms, dev)
+        g_ms, g_host_us = time_graph(prob, args.steps, args.warmup, flush, stream)
+        g_ms = max_over_ranks(g_ms, dev)
+        h_host_us = host_call_us(prob, 20, stream)
         metric, unit = metric_of(name)
         line = {"metric": metric, "value": value_of(name, work, ms, n), "unit": unit,
                 "ms_per_step": ms,
@@ -448,7 +517,10 @@ def main():
                 "e2e": {"value": value_of(name, work, e2e_ms, n), "unit": unit,
                         "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},
-                "gpu_launches": int(sum(v[0] for v in kern.values()))}
+                "gpu_launches": int(sum(v[0] for v in kern.values())),
+                "device_planned_graph": {"value": value_of(name, work, g_ms, n), "unit": unit,
+                                         "ms_per_step": g_ms, "host_us_per_replay": g_host_us,
+                                         "host_us_per_host_planned_call": h_host_us}}
         if rank == 0 and i == 0 and world == 1:
             cpu_base = cpu_baseline(name, prob, args.cpu_budget)
         results.append(line)
@@ -463,6 +535,7 @@ def main():
                "config": {**head["config"], "parallelism": f"replicas x{n}" if n > 1 else "1 GPU"},
                "roofline": head["roofline"], "e2e": head["e2e"],
                "gpu_launches": head["gpu_launches"], "clocks": clk,
+               "device_planned_graph": head["device_planned_graph"],
                "cpu_baseline": cpu_base, "also": results[1:]}
         print(json.dumps(out), flush=True)
     if world > 1:

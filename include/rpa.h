@@ -312,8 +312,10 @@ RPA_API int rpa_device_workspace_size(const rpa_dims *dims, int32_t max_seqs,
  *     and arguments depend only on the pointers, dims, max_seqs, scale,
  *     causal and the option values, never on the lengths: the host neither
  *     reads device memory nor waits, so the call can be captured into a CUDA
- *     graph and replayed.  The head_dim <= 128 prefill kernel takes one TMA
- *     producer warp for K and V unless RPA_OPT_PREFILL_LOADERS is 2.
+ *     graph and replayed.  The planner kernel makes the per-batch choices
+ *     rpa_forward's host planner makes (packing of short decode sequences,
+ *     the producer layout of the head_dim <= 128 prefill kernel) by the same
+ *     rules, from the device-resident lengths.
  * Results (out, lse, cache contents) are those rpa_forward gives for the same
  * batch.  max_seqs == 0 or T == 0 is a successful no-op.  Host-side checks
  * (scale, dims, null pointers, workspace) return RPA_ERR_* before anything is

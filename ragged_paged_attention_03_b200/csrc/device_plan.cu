@@ -91,7 +91,7 @@ DeviceLayout device_layout(const rpa_dims *d, int32_t max_seqs) {
 
 struct PlanArgs {
   const int32_t *cu, *kv, *num_seqs;
-  int32_t max_seqs, T, P, max_pages, hkv, chunk, pack, item_rows, bf16;
+  int32_t max_seqs, T, P, max_pages, hkv, chunk, pack, item_rows, bf16, loaders;
   int32_t *counts;
   uint32_t *err;
   DecodeItem *items, *packed;
@@ -124,7 +124,7 @@ __device__ int offsets_largest_first(int *h, int nb, int lane) {
 }
 
 __device__ __forceinline__ void write_counts(int32_t *counts, int dec, int packed, int comb, int tiles,
-                                             int gseqs, int grows, int partials) {
+                                             int gseqs, int grows, int partials, int split) {
   counts[kCntDecode] = dec;
   counts[kCntPacked] = packed;
   counts[kCntCombine] = comb;
@@ -132,16 +132,20 @@ __device__ __forceinline__ void write_counts(int32_t *counts, int dec, int packe
   counts[kCntGenericSeqs] = gseqs;
   counts[kCntGenericRows] = grows;
   counts[kCntPartials] = partials;
-  counts[7] = 0;
+  counts[kCntPrefillSplit] = split;
 }
 
 __global__ void __launch_bounds__(kPlanThreads) device_plan_kernel(const PlanArgs a) {
   __shared__ int h_items[kLenBins], h_packed[kLenBins], h_tiles[kTileBins];
   __shared__ int s_short, s_partials, s_combine, s_total[3];
+  __shared__ unsigned long long s_ctx, s_new;   // prefill rows: cached context, new tokens
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int i = tid; i < kLenBins; i += kPlanThreads) h_items[i] = h_packed[i] = 0;
   for (int i = tid; i < kTileBins; i += kPlanThreads) h_tiles[i] = 0;
-  if (tid == 0) s_short = s_partials = s_combine = 0;
+  if (tid == 0) {
+    s_short = s_partials = s_combine = 0;
+    s_ctx = s_new = 0;
+  }
 
   // ---- validation (the host path's rules) and the count of packable sequences
   int n = *a.num_seqs;
@@ -163,7 +167,7 @@ __global__ void __launch_bounds__(kPlanThreads) device_plan_kernel(const PlanArg
   if (my_short) atomicAdd(&s_short, my_short);
   if (__syncthreads_or(bad)) {
     if (tid == 0) {
-      write_counts(a.counts, 0, 0, 0, 0, 0, 0, 0);
+      write_counts(a.counts, 0, 0, 0, 0, 0, 0, 0, 0);
       atomicOr(a.err, RPA_DEV_BAD_LENGTHS);
     }
     return;
@@ -180,13 +184,14 @@ __global__ void __launch_bounds__(kPlanThreads) device_plan_kernel(const PlanArg
       g.row_prefix = a.cu[s];
       a.generic[s] = g;
     }
-    if (tid == 0) write_counts(a.counts, 0, 0, 0, 0, n, a.cu[n], 0);
+    if (tid == 0) write_counts(a.counts, 0, 0, 0, 0, n, a.cu[n], 0, 0);
     return;
   }
 
   const bool packing = a.pack > 0 && (int64_t)((s_short + 3) / 4) * a.hkv >= kMinPackedCtas;
   const int R = a.item_rows;
   // ---- histograms of the sort keys
+  unsigned long long my_ctx = 0, my_new = 0;
   for (int s = tid; s < n; s += kPlanThreads) {
     const int ql = a.cu[s + 1] - a.cu[s], kvl = a.kv[s];
     if (ql == 1) {
@@ -199,11 +204,17 @@ __global__ void __launch_bounds__(kPlanThreads) device_plan_kernel(const PlanArg
         atomicAdd(&h_items[nb - (ns - 1) * per], 1);
       }
     } else if (ql > 1) {
+      my_ctx += (unsigned long long)(kvl - ql);
+      my_new += (unsigned long long)ql;
       for (int r = 0; r < ql; r += R) {
         const int w = kvl - ql + r + min(R, ql - r);   // keys visible to the tile's last row
         atomicAdd(&h_tiles[min(w >> 7, kTileBins - 1)], 1);
       }
     }
+  }
+  if (my_new) {
+    atomicAdd(&s_ctx, my_ctx);
+    atomicAdd(&s_new, my_new);
   }
   __syncthreads();
   if (warp == 0) {
@@ -220,7 +231,7 @@ __global__ void __launch_bounds__(kPlanThreads) device_plan_kernel(const PlanArg
   // the capacities bound these by construction; a mismatch writes nothing
   if (s_total[0] > a.cap_items || s_total[1] > a.cap_packed || s_total[2] > a.cap_tiles) {
     if (tid == 0) {
-      write_counts(a.counts, 0, 0, 0, 0, 0, 0, 0);
+      write_counts(a.counts, 0, 0, 0, 0, 0, 0, 0, 0);
       atomicOr(a.err, RPA_DEV_BAD_LENGTHS);
     }
     return;
@@ -274,8 +285,13 @@ __global__ void __launch_bounds__(kPlanThreads) device_plan_kernel(const PlanArg
       }
     }
   }
+  // empty tiles after the last one end the persistent prefill kernel's list
+  for (int64_t i = s_total[2] + tid; i < a.cap_tiles; i += kPlanThreads) a.tiles[i] = PrefillTile{};
   __syncthreads();
-  if (tid == 0) write_counts(a.counts, s_total[0], s_total[1], s_combine, s_total[2], 0, 0, s_partials);
+  // producer layout of the head_dim <= 128 prefill kernel, the host planner's
+  // rule: one warp per operand when the prefill rows are mostly cached context
+  const int split = a.loaders == 2 || (a.loaders != 1 && s_ctx > s_new);
+  if (tid == 0) write_counts(a.counts, s_total[0], s_total[1], s_combine, s_total[2], 0, 0, s_partials, split);
 }
 
 }  // namespace
@@ -329,6 +345,7 @@ extern "C" RPA_API int rpa_forward_device(const void *q, const void *k_new, cons
   a.pack = L.pack;
   a.item_rows = prefill_item_rows(dims->head_dim);
   a.bf16 = dims->dtype == RPA_BF16 ? 1 : 0;
+  a.loaders = (int32_t)prefill_loaders();
   a.counts = counts;
   a.err = dev_flags ? dev_flags : reinterpret_cast<uint32_t *>(ws + kErrOffset);
   a.items = reinterpret_cast<DecodeItem *>(ws + L.items);
@@ -374,7 +391,7 @@ extern "C" RPA_API int rpa_forward_device(const void *q, const void *k_new, cons
     if (e == cudaSuccess && L.cap_combine > 0)
       e = launch_combine(pb, a.combine, (int)L.cap_combine, part_o, part_lse, stream);
     if (e == cudaSuccess && L.cap_tiles > 0)
-      e = pb.d <= 128 ? launch_prefill2(pb, a.tiles, (int)L.cap_tiles, 0, prefill_loaders() == 2, stream)
+      e = pb.d <= 128 ? launch_prefill2(pb, a.tiles, (int)L.cap_tiles, 0, false, stream)
                       : launch_prefill(pb, a.tiles, (int)L.cap_tiles, stream);
   } else if (e == cudaSuccess) {
     e = launch_generic(pb, a.generic, max_seqs, dims->total_q_tokens, stream);

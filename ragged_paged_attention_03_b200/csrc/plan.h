@@ -64,7 +64,8 @@ struct PrefillTile {
 // Device-planned calls (rpa_forward_device): the planner kernel writes the
 // work counts into a header of int32 slots; each kernel of the call is
 // launched with a grid sized for the workspace's capacity and bounds its work
-// by its slot.  Host-planned calls pass no header.
+// by its slot (the persistent head_dim <= 128 prefill kernel by an empty tile,
+// rows == 0, after the last one).  Host-planned calls pass no header.
 enum DeviceCount {
   kCntDecode = 0,       // decode work items
   kCntPacked = 1,       // packed (four per CTA) decode items
@@ -73,6 +74,8 @@ enum DeviceCount {
   kCntGenericSeqs = 4,  // generic-kernel sequences
   kCntGenericRows = 5,  // generic-kernel rows
   kCntPartials = 6,     // split-KV partial slots in use
+  kCntPrefillSplit = 7, // 1: the head_dim <= 128 prefill kernel gives K and V
+                        // a producer warp each (its split build)
   kCntSlots = 8
 };
 

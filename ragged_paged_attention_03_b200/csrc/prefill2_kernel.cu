@@ -14,8 +14,8 @@
 //   warp 9                   TMEM owner and MMA issue
 //   warps 10-11              fused cache update: this CTA's share of the new
 //                            K/V rows copied into their page slots
-// A second build of the kernel (SPLIT) gives V a producer of its own in warp
-// 10, leaving warp 11 to the cache update: the planner picks it for batches
+// A second role layout (the `split` argument) gives V a producer of its own in
+// warp 10, leaving warp 11 to the cache update: the planner picks it for batches
 // whose prefill work is mostly paged context (latency-bound gathers, few new
 // rows to write), the first one otherwise.
 // The producer and MMA warps run their loops with all 32 lanes and let one
@@ -204,6 +204,7 @@ __device__ __forceinline__ void mma_loop(Bars2 *bars, volatile int *abort_flag, 
   bool ok = true;
   for (int r = 0, u = unit_of(0); ok && u < n_units; u = unit_of(++r), ++uq) {
     const Unit w = make_unit<BM, BN>(tiles, u, pb);
+    if (w.tile.rows == 0) break;   // end of a device-planned tile list
     const int n0 = w.n_t[0], n1 = w.n_t[1], nb = w.nb;
     ok = wait_all(&bars->q_full, (uint32_t)(uq & 1), abort_flag, err);
     // prologue
@@ -282,6 +283,7 @@ __device__ __forceinline__ void produce_kv(Bars2 *bars, volatile int *abort_flag
   bool ok = true;
   for (int r = 0, u = unit_of(0); ok && u < n_units; u = unit_of(++r), ++uq) {
     const Unit w = make_unit<BM, BN>(tiles, u, pb);
+    if (w.tile.rows == 0) break;   // end of a device-planned tile list
     const int32_t *pt_row = pb.page_table + (size_t)w.tile.seq * pb.max_pages;
     // Q of both tiles, once the previous unit's QK MMAs are done with sQ
     if (uq > 0 && !wait_all(&bars->q_empty, (uint32_t)((uq - 1) & 1), abort_flag, pb.err)) break;
@@ -435,6 +437,7 @@ __device__ __forceinline__ void produce(Bars2 *bars, volatile int *abort_flag, c
   bool ok = true;
   for (int r = 0, u = unit_of(0); ok && u < n_units; u = unit_of(++r), ++uq) {
     const Unit w = make_unit<BM, BN>(tiles, u, pb);
+    if (w.tile.rows == 0) break;   // end of a device-planned tile list
     const int32_t *pt_row = pb.page_table + (size_t)w.tile.seq * pb.max_pages;
     if (!IS_V) {
       // Q of both tiles, once the previous unit's QK MMAs are done with sQ
@@ -545,6 +548,7 @@ __device__ __forceinline__ void cache_update(const Problem pb, const PrefillTile
   __nv_bfloat16 *vc = reinterpret_cast<__nv_bfloat16 *>(pb.v_cache);
   for (int r = 0, u = unit_of(0); u < n_units; u = unit_of(++r)) {
     const Unit w = make_unit<BM, BN>(tiles, u, pb);
+    if (w.tile.rows == 0) break;   // end of a device-planned tile list
     const int32_t *pt_row = pb.page_table + (size_t)w.tile.seq * pb.max_pages;
     const int gidx = w.h % G;
     const int ra = (gidx * w.tile.rows) / G, rb = ((gidx + 1) * w.tile.rows) / G;
@@ -572,15 +576,16 @@ __device__ __forceinline__ void cache_update(const Problem pb, const PrefillTile
 // Every barrier parity runs on counters that span units, so the producer
 // loads the next unit's Q and K/V while the current one finishes and the MMA
 // warp starts the next unit while the softmax warps are still storing O.
-// DEV: a device-planned call (capacity-sized grid, the unit count read from
-// pb.dev_counts); a separate instance so that the host-planned build keeps
-// its count in the kernel parameters rather than in a register.
-template <int D, bool SPLIT, bool DEV>
+// split: V gets a producer warp of its own (warp 10) and the cache update
+// one warp (11); otherwise warp 8 loads K and V and warps 10-11 update the
+// cache.  A device-planned call passes the capacity's unit count; the
+// planner ends the tile list with empty tiles and chooses split.
+template <int D>
 __global__ void __launch_bounds__(384, 1)
     prefill2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
                     const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_kn,
                     const __grid_constant__ CUtensorMap tm_vn, const Problem pb,
-                    const PrefillTile *__restrict__ tiles, int n_units, float scale_log2) {
+                    const PrefillTile *__restrict__ tiles, int n_units, int split, float scale_log2) {
   using S = P2Shape<D>;
   constexpr int BM = S::BM, BN = S::BN, NSK = S::NSK, NSV = S::NSV;
   extern __shared__ uint8_t smem_raw[];
@@ -595,10 +600,10 @@ __global__ void __launch_bounds__(384, 1)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  if (DEV) {
+  if (pb.dev_counts != nullptr) {
     // capacity-sized grid: CTAs without a unit leave before any set-up
-    n_units = min(n_units, pb.dev_counts[kCntPrefill] * pb.hq);
-    if ((int)blockIdx.x >= n_units) return;
+    if ((int)blockIdx.x >= pb.dev_counts[kCntPrefill] * pb.hq) return;
+    split = pb.dev_counts[kCntPrefillSplit];
   }
 
   if (tid == 0) {
@@ -644,7 +649,7 @@ __global__ void __launch_bounds__(384, 1)
   if (warp >= 8) {
     setmaxnreg_dec96();
     if (warp == 8) {
-      if (SPLIT)
+      if (split)
         produce<D, false>(bars, abort_flag, pb, tiles, n_units, sQ, sK, &tm_q, &tm_kn, &tm_kc);
       else
         produce_kv<D>(bars, abort_flag, pb, tiles, n_units, sQ, sK, sV, &tm_q, &tm_kc, &tm_vc, &tm_kn, &tm_vn);
@@ -652,11 +657,11 @@ __global__ void __launch_bounds__(384, 1)
       // --------------------------------------------------------------- MMA
       mma_loop<D>(bars, abort_flag, pb, tiles, n_units, tmem, ptx::smem_u32(sQ), ptx::smem_u32(sK),
                   ptx::smem_u32(sV));
-    } else if (SPLIT && warp == 10) {
+    } else if (split && warp == 10) {
       produce<D, true>(bars, abort_flag, pb, tiles, n_units, sQ, sV, &tm_q, &tm_vn, &tm_vc);
     } else {
       // fused cache update: warps 10-11, or warp 11 when warp 10 loads V
-      cache_update<D>(pb, tiles, n_units, SPLIT ? lane : tid - 320, SPLIT ? 32 : 64);
+      cache_update<D>(pb, tiles, n_units, split ? lane : tid - 320, split ? 32 : 64);
     }
   } else {
     // ----------------------------------------------------------- softmax
@@ -671,6 +676,7 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
     for (int r = 0, u = unit_of(0); ok && u < n_units; u = unit_of(++r)) {
       const Unit w = make_unit<BM, BN>(tiles, u, pb);
+      if (w.tile.rows == 0) break;   // end of a device-planned tile list
       // tile-uniform selects keep the unit in registers (no local memory)
       const int n = t ? w.n_t[1] : w.n_t[0];
       const int rows_mine = t ? w.rows_t[1] : w.rows_t[0];
@@ -830,9 +836,7 @@ cudaError_t launch_t(const Problem &pb, const PrefillTile *tiles, int n_tiles, i
       !make_tmap_bf16_3d(&tkn, pb.k_new, ndims, nstr, nbox, true) ||
       !make_tmap_bf16_3d(&tvn, pb.v_new, ndims, nstr, nbox, true))
     return cudaErrorInvalidValue;
-  const bool dev = pb.dev_counts != nullptr;
-  auto kern = split ? (dev ? prefill2_kernel<D, true, true> : prefill2_kernel<D, true, false>)
-                    : (dev ? prefill2_kernel<D, false, true> : prefill2_kernel<D, false, false>);
+  auto kern = prefill2_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem);
   if (e != cudaSuccess) return e;
   const int n_units = n_tiles * pb.hq;
@@ -845,7 +849,8 @@ cudaError_t launch_t(const Problem &pb, const PrefillTile *tiles, int n_tiles, i
   }
   int grid = n_units < sms ? n_units : sms;
   if (max_ctas > 0 && grid > max_ctas) grid = max_ctas;
-  kern<<<grid, 384, S::kSmem, stream>>>(tq, tkc, tvc, tkn, tvn, pb, tiles, n_units, pb.scale * kLog2e);
+  kern<<<grid, 384, S::kSmem, stream>>>(tq, tkc, tvc, tkn, tvn, pb, tiles, n_units, split ? 1 : 0,
+                                        pb.scale * kLog2e);
   return cudaGetLastError();
 }
 
