@@ -285,7 +285,7 @@ RPA_API int rpa_device_workspace_size(const rpa_dims *dims, int32_t max_seqs,
 /*
  * rpa_forward_device -- rpa_forward with the metadata pass on the GPU, for
  * CUDA-graph capture.  The pages propose moving the kernel's scalar metadata
- * work off the main compute path (arXiv 2604.15464, future work: SparseCore
+ * work off the main compute path (talk summary 00:16:06 and 00:18:14: SparseCore
  * offload); here a one-CTA planner kernel, queued on `stream` before the
  * attention kernels, reads the lengths from device memory and writes the
  * work lists into `workspace`.

@@ -9,8 +9,9 @@
 //   blocks of one sequence; long sequences are cut into several items whose
 //   partial results the combine kernel merges (log-sum-exp weighting).
 // * Short sequences are packed instead: four whole-sequence items per CTA,
-//   one per warp, each warp streaming all of its item's blocks (the pages'
-//   fix for requests too short to fill the bandwidth on their own).
+//   one per warp, each warp streaming all of its item's blocks (the
+//   multi-request batching the talk's roadmap, 00:18:14, proposes for
+//   sequences too short to fill the bandwidth on their own).
 // * The CTA's four warps stream disjoint blocks (block b goes to warp
 //   b mod 4), each with its own ring of shared-memory stages fed by TMA
 //   (cp.async.bulk.tensor, 128-byte swizzle, one 16-row box per page part

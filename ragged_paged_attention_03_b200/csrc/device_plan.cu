@@ -4,7 +4,8 @@
 //
 // The pages propose moving the kernel's scalar metadata work (sequence
 // bookkeeping, tile boundaries) off the main compute path, to the TPU's
-// SparseCore ("Ragged Paged Attention", arXiv 2604.15464, future work).  On
+// SparseCore (RPA talk summary, rocketrecap.com, 00:16:06 and the roadmap
+// at 00:18:14).  On
 // B200 the counterpart is a one-CTA planner kernel on the same stream: it
 // reads cu_q_lens / kv_lens / num_seqs from device memory, validates them,
 // routes every sequence (decode: one new token; prefill / chunked prefill:
