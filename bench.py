@@ -491,11 +491,22 @@ def main():
         if world > 1:
             torch.distributed.barrier()
         torch.cuda.synchronize(dev)
+        # a batch with prefill and decode rows runs them concurrently (two
+        # streams); its per-kernel event times overlap, so the kernel
+        # rooflines of such a step come from a serial run of the same step
+        mixed = work["prefill_flops"] > 0 and work["decode_kernel_bytes"] > 0
         if i == 0:
             clocks.start()
-        ms, kern = time_steps(prob, args.steps, args.warmup, flush, stream, profile=True)
+        ms, kern = time_steps(prob, args.steps, args.warmup, flush, stream, profile=not mixed)
         if i == 0:
             clk = clocks.stop()
+        if mixed:
+            from ragged_paged_attention_03_b200 import binding as rb
+            old = rb.rpa_set_option(rb.RPA_OPT_CONCURRENT_MIXED, -1)
+            try:
+                serial_ms, kern = time_steps(prob, args.steps, args.warmup, flush, stream, profile=True)
+            finally:
+                rb.rpa_set_option(rb.RPA_OPT_CONCURRENT_MIXED, old)
         torch.cuda.synchronize(dev)
         ms = max_over_ranks(ms, dev)
         if world > 1:
@@ -513,7 +524,10 @@ def main():
                            "l2": "flushed between steps (256 MiB write)",
                            "tokens": work["tokens"], "bytes": work["bytes"],
                            "flops": work["flops"]},
-                "roofline": roofline(name, work, kern, pk, args.steps),
+                "roofline": {**roofline(name, work, kern, pk, args.steps),
+                             **({"kernel_timing": f"serial run of the same step ({serial_ms:.4f} ms), "
+                                                  "since the step itself runs prefill and decode concurrently"}
+                                if mixed else {})},
                 "e2e": {"value": value_of(name, work, e2e_ms, n), "unit": unit,
                         "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},

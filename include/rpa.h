@@ -192,14 +192,15 @@ enum {
                                       kernel (default 0) */
   RPA_OPT_DISABLE_PREFILL_TC = 2,  /* 1: prefill sequences use the generic
                                       kernel instead of tensor cores */
-  RPA_OPT_PREFILL_SMS = 3,         /* SMs given to the prefill kernel when
-                                      RPA_OPT_CONCURRENT_MIXED is on (0 =
-                                      chosen from the batch's estimated FLOPs
-                                      and bytes) */
-  RPA_OPT_CONCURRENT_MIXED = 4,    /* 1: run the prefill and decode work of a
-                                      mixed batch concurrently on two streams
-                                      (default 0: one after the other, faster
-                                      on the measured mixes) */
+  RPA_OPT_PREFILL_SMS = 3,         /* most CTAs (SMs) of the head_dim <= 128
+                                      prefill kernel in a concurrent mixed
+                                      batch (default 0: one per SM) */
+  RPA_OPT_CONCURRENT_MIXED = 4,    /* >= 0 (default 0): the prefill and the
+                                      decode work of a mixed batch run
+                                      concurrently, prefill on a
+                                      highest-priority library stream that the
+                                      caller's stream joins before the call
+                                      returns; < 0: one after the other */
   RPA_OPT_PREFILL_LOADERS = 5,     /* TMA producer warps of the head_dim <= 128
                                       prefill kernel: 1 (K and V share one), 2
                                       (one each; the cache update gets one warp

@@ -24,6 +24,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "host_common.h"
 #include "kernels.h"
@@ -40,6 +41,30 @@ constexpr int64_t kAlign = 256;
 constexpr int64_t kErrOffset = 128;                  // error word in the header
 
 int64_t align_up(int64_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// Per device: the highest-priority stream the prefill kernel runs on, next
+// to the decode kernels on the caller's stream, and the fork / join events.
+// Captured into a graph these become two parallel branches.
+struct SideStream {
+  std::mutex mu;
+  bool init = false;
+  cudaStream_t side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kMaxDevices = 64;
+SideStream g_side[kMaxDevices];
+
+bool side_init(SideStream &s) {
+  if (s.init) return true;
+  int lo = 0, hi = 0;
+  if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess) hi = 0;
+  if (cudaStreamCreateWithPriority(&s.side, cudaStreamNonBlocking, hi) != cudaSuccess ||
+      cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming) != cudaSuccess)
+    return false;
+  s.init = true;
+  return true;
+}
 
 // Capacities and byte offsets of a device-planned call's workspace.  Every
 // bound follows from the geometry alone: a decode sequence takes one new
@@ -385,15 +410,37 @@ extern "C" RPA_API int rpa_forward_device(const void *q, const void *k_new, cons
   float *part_o = reinterpret_cast<float *>(ws + L.part_o);
   float *part_lse = reinterpret_cast<float *>(ws + L.part_lse);
   if (dims->dtype == RPA_BF16) {
+    // prefill and decode concurrently, as rpa_forward runs a mixed batch:
+    // prefill on the highest-priority side stream (its CTAs are placed
+    // first), decode on the caller's stream filling the SMs prefill leaves
+    const bool both = L.cap_tiles > 0 && L.cap_items > 0 && concurrent_mixed();
+    SideStream *ss = nullptr;
+    std::unique_lock<std::mutex> lock;
+    cudaStream_t pstream = stream;
+    if (e == cudaSuccess && both) {
+      int dev = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RPA_ERR_CUDA;
+      ss = &g_side[dev];
+      lock = std::unique_lock<std::mutex>(ss->mu);
+      if (!side_init(*ss)) return RPA_ERR_CUDA;
+      if (cudaEventRecord(ss->fork, stream) != cudaSuccess || cudaStreamWaitEvent(ss->side, ss->fork, 0) != cudaSuccess)
+        return RPA_ERR_CUDA;
+      pstream = ss->side;
+    }
+    if (e == cudaSuccess && L.cap_tiles > 0)
+      e = pb.d <= 128 ? launch_prefill2(pb, a.tiles, (int)L.cap_tiles, (int)prefill_sms(), false, pstream)
+                      : launch_prefill(pb, a.tiles, (int)L.cap_tiles, pstream);
+    const cudaError_t ej = ss ? cudaEventRecord(ss->join, pstream) : cudaSuccess;
+    if (e == cudaSuccess) e = ej;
     if (e == cudaSuccess && L.cap_items > 0)
       e = launch_decode(pb, a.items, (int)L.cap_items, part_o, part_lse, false, stream);
     if (e == cudaSuccess && L.cap_packed > 0)
       e = launch_decode(pb, a.packed, (int)L.cap_packed, part_o, part_lse, true, stream);
     if (e == cudaSuccess && L.cap_combine > 0)
       e = launch_combine(pb, a.combine, (int)L.cap_combine, part_o, part_lse, stream);
-    if (e == cudaSuccess && L.cap_tiles > 0)
-      e = pb.d <= 128 ? launch_prefill2(pb, a.tiles, (int)L.cap_tiles, 0, false, stream)
-                      : launch_prefill(pb, a.tiles, (int)L.cap_tiles, stream);
+    // join (also after an error, so that nothing of the call runs unordered)
+    if (ss && ej == cudaSuccess && cudaStreamWaitEvent(stream, ss->join, 0) != cudaSuccess && e == cudaSuccess)
+      e = cudaErrorUnknown;
   } else if (e == cudaSuccess) {
     e = launch_generic(pb, a.generic, max_seqs, dims->total_q_tokens, stream);
   }

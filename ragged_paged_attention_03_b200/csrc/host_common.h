@@ -15,6 +15,8 @@ int validate_dims(const rpa_dims *d);
 int64_t decode_chunk_blocks();   // 16-token blocks per decode work item
 int64_t decode_pack_blocks();    // longest packed decode sequence, 0 = never
 int64_t prefill_loaders();       // RPA_OPT_PREFILL_LOADERS as set (0, 1, 2)
+bool concurrent_mixed();         // RPA_OPT_CONCURRENT_MIXED >= 0
+int64_t prefill_sms();           // RPA_OPT_PREFILL_SMS (<= 0: one CTA per SM)
 
 // Packed decode CTAs a batch must fill before packing is used (two per SM
 // of a 148-SM B200): a packed launch follows the main decode launch, so a

@@ -60,6 +60,10 @@ int64_t decode_pack_blocks() {
 
 int64_t prefill_loaders() { return g_opt_prefill_loaders.load(); }
 
+bool concurrent_mixed() { return g_opt_concurrent_mixed.load() >= 0; }
+
+int64_t prefill_sms() { return g_opt_prefill_sms.load(); }
+
 int validate_dims(const rpa_dims *d) {
   if (d == nullptr) return RPA_ERR_INVALID_ARG;
   if (d->num_q_heads <= 0 || d->num_kv_heads <= 0 || d->num_pages <= 0 ||
@@ -323,7 +327,12 @@ int ensure_init(DeviceWs &ws) {
         cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming) != cudaSuccess)
       return RPA_ERR_CUDA;
-  if (cudaStreamCreateWithFlags(&ws.side, cudaStreamNonBlocking) != cudaSuccess) return RPA_ERR_CUDA;
+  // the side stream runs the prefill of a concurrent mixed batch: the
+  // highest priority makes the block scheduler place its (whole-SM) CTAs
+  // before the decode kernel's, which then fill each SM as it frees
+  int lo_prio = 0, hi_prio = 0;
+  if (cudaDeviceGetStreamPriorityRange(&lo_prio, &hi_prio) != cudaSuccess) hi_prio = 0;
+  if (cudaStreamCreateWithPriority(&ws.side, cudaStreamNonBlocking, hi_prio) != cudaSuccess) return RPA_ERR_CUDA;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&ws.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || ws.sms <= 0)
@@ -525,24 +534,19 @@ extern "C" RPA_API int rpa_forward(const void *q, const void *k_new, const void 
     float *partial_o = slot.partial;
     float *partial_lse = slot.partial ? slot.partial + L.n_partials * dims->num_kv_heads * G * dims->head_dim : nullptr;
     cudaError_t e = cudaSuccess;
-    // Optionally, a batch with both prefill and decode work runs them
-    // concurrently: the compute-bound prefill kernel on the side stream with a
-    // share of the SMs, the bandwidth-bound decode kernel on the caller's
-    // stream on the rest.
+    // A batch with both prefill and decode work runs them concurrently: the
+    // compute-bound prefill kernel on the high-priority side stream, queued
+    // first, takes the SMs (one whole-SM CTA each); the bandwidth-bound decode
+    // kernel on the caller's stream fills every SM its prefill CTA leaves, so
+    // the prefill's uneven finish is covered instead of waited for.
     const bool mixed = L.n_prefill_tiles > 0 &&
                        (L.n_decode_items > 0 || L.n_decode_packed > 0 || L.n_generic_rows > 0) &&
-                       g_opt_concurrent_mixed.load() != 0;
+                       g_opt_concurrent_mixed.load() >= 0;
     cudaStream_t pstream = stream;
     int prefill_ctas = 0;
     if (mixed) {
-      int64_t k = g_opt_prefill_sms.load();
-      if (k <= 0) {
-        // balance the two finishing times: prefill at ~0.9 PFLOP/s and decode
-        // at ~5.5 TB/s when each has the whole GPU
-        const double tp = hp.prefill_flops / 0.9e15, td = hp.decode_bytes / 5.5e12;
-        k = (int64_t)(ws.sms * (tp / (tp + td + 1e-30)) + 0.5);
-      }
-      prefill_ctas = (int)std::max<int64_t>(8, std::min<int64_t>(k, ws.sms - 8));
+      const int64_t k = g_opt_prefill_sms.load();
+      prefill_ctas = k > 0 ? (int)std::min<int64_t>(k, ws.sms) : 0;   // 0: one per SM
       pstream = ws.side;
       if (cudaEventRecord(slot.fork, stream) != cudaSuccess || cudaStreamWaitEvent(pstream, slot.fork, 0) != cudaSuccess)
         return RPA_ERR_CUDA;

@@ -116,6 +116,20 @@ def test_more_shapes(oracle_mod, case):
     one_shot(oracle_mod, prob)
 
 
+def test_serial_schedule(oracle_mod):
+    """RPA_OPT_CONCURRENT_MIXED < 0: the device-planned call queues every
+    kernel on the caller's stream (no side-stream branch)."""
+    from ragged_paged_attention_03_b200 import binding as rb
+    ql, kv, hq, hkv, d, p, causal = SMALL[6]
+    prob = I.make_problem(ql, kv, num_q_heads=hq, num_kv_heads=hkv, head_dim=d, page_size=p,
+                          dtype=I.BF16, causal=causal, seed=990, pool=1.5, name="dev-serial")
+    old = rb.rpa_set_option(rb.RPA_OPT_CONCURRENT_MIXED, -1)
+    try:
+        one_shot(oracle_mod, prob)
+    finally:
+        rb.rpa_set_option(rb.RPA_OPT_CONCURRENT_MIXED, old)
+
+
 def test_split_kv_and_packed_decode(oracle_mod):
     """Enough short decode sequences to be packed four per CTA, next to long
     ones cut into chunks (1-block chunks force many partials)."""

@@ -79,13 +79,16 @@ def test_without_distribution_and_shuffled_order(oracle_mod):
     full_check(oracle_mod, prob, use_distribution=False)
 
 
-def test_concurrent_mixed_batch(oracle_mod):
-    """The opt-in concurrent execution of a mixed batch (prefill on a second
-    stream with a share of the SMs, decode on the caller's stream) gives the
-    oracle's results too."""
+@pytest.mark.parametrize("concurrent,sms", [(1, 20), (-1, 0)])
+def test_mixed_batch_schedules(oracle_mod, concurrent, sms):
+    """A mixed batch with its prefill kernel limited to 20 CTAs on the side
+    stream (decode on the caller's stream around it), and the same batch run
+    one kernel after the other (RPA_OPT_CONCURRENT_MIXED < 0): both give the
+    oracle's results (the default, concurrent on every SM, runs in the other
+    mixed tests)."""
     from ragged_paged_attention_03_b200 import binding
-    old_c = binding.rpa_set_option(binding.RPA_OPT_CONCURRENT_MIXED, 1)
-    old_k = binding.rpa_set_option(binding.RPA_OPT_PREFILL_SMS, 20)
+    old_c = binding.rpa_set_option(binding.RPA_OPT_CONCURRENT_MIXED, concurrent)
+    old_k = binding.rpa_set_option(binding.RPA_OPT_PREFILL_SMS, sms)
     try:
         prob = I.make_problem([1] * 6 + [300, 77], [40, 900, 2100, 1, 17, 300, 300, 500],
                               num_q_heads=32, num_kv_heads=8, head_dim=128, page_size=16,
