@@ -206,15 +206,14 @@ __global__ void __launch_bounds__(192, 1)
           for (int hh = 0; hh < S::kHalves; ++hh)
             ptx::tma_load_3d_elect(dst + hh * BN * 128, tm_new, bar, hh * 64, hk, row);
         } else {
-          // every lane takes part in the broadcast of segment sg's page id
-          for (int sg = 0; sg < nseg; ++sg) {
-            const int pg = __shfl_sync(0xffffffffu, page, sg);
-            if (!((loaded_mask >> sg) & 1u)) continue;
-            const int sp = pos0 + sg * br;
-            const int row = pg * pb.p + (sp % pb.p);
+          // each lane queues the copies of its own page segment, so one
+          // instruction covers every segment of the block
+          if ((loaded_mask >> lane) & 1u) {
+            const int row = page * pb.p + ((pos0 + lane * br) % pb.p);
             for (int hh = 0; hh < S::kHalves; ++hh)
-              ptx::tma_load_3d_elect(dst + hh * BN * 128 + sg * br * 128, tm_ctx, bar, hh * 64, hk, row);
+              ptx::tma_load_3d(dst + hh * BN * 128 + lane * br * 128, tm_ctx, bar, hh * 64, hk, row);
           }
+          __syncwarp();
         }
       };
       if (!fix) {
