@@ -164,8 +164,9 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ GPU arm
-def device_problem(name: str, causal, device, max_seqs=None) -> I.Problem:
-    return I.make_workload(name, device=device, causal=causal, poison=False, max_seqs=max_seqs)
+def device_problem(name: str, causal, device, max_seqs=None, head_shard=None) -> I.Problem:
+    return I.make_workload(name, device=device, causal=causal, poison=False, max_seqs=max_seqs,
+                           head_shard=head_shard)
 
 
 def time_steps(prob, steps, warmup, flush, stream, profile=False):
@@ -319,6 +320,17 @@ def metric_of(name):
     return "long-context HBM GB/s", "GB/s"
 
 
+def rank_work(work: dict, world: int, shard: str) -> dict:
+    """One rank's share of the job's work, as value_of counts it (value =
+    world x a rank's share / time).  Replicas: each rank does the whole
+    batch.  KV-head shards: bytes and FLOPs split over the ranks, but every
+    rank serves all the batch's tokens (for its heads), so its share of the
+    job's tokens is tokens / world."""
+    if shard != "heads" or world == 1:
+        return work
+    return {**work, "tokens": work["tokens"] / world}
+
+
 def value_of(name, work, ms, n):
     metric, unit = metric_of(name)
     if unit == "GB/s":
@@ -437,6 +449,9 @@ def main():
                     help="seconds of oracle work for the cpu_baseline sample")
     ap.add_argument("--max-seqs", type=int, default=None,
                     help="keep only the first N sequences of each workload (profiler captures)")
+    ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
+                    help="replicas: every GPU runs the whole batch (weak scaling); heads: every GPU "
+                         "runs its Hkv/N KV heads of the same batch (strong scaling; no collective)")
     args = ap.parse_args()
     world, rank, local = dist_setup(args)
     n = world
@@ -486,8 +501,9 @@ def main():
     for i, spec in enumerate(wl):
         name, _, opt = spec.partition(":")
         causal = False if opt == "noncausal" else None
-        prob = device_problem(name, causal, dev, args.max_seqs)
-        work = algorithmic(prob)
+        prob = device_problem(name, causal, dev, args.max_seqs,
+                              head_shard=(rank, world) if args.shard == "heads" else None)
+        work = rank_work(algorithmic(prob), world, args.shard)
         if world > 1:
             torch.distributed.barrier()
         torch.cuda.synchronize(dev)
@@ -544,9 +560,12 @@ def main():
         head = results[0]
         out = {"metric": head["metric"], "value": head["value"], "unit": head["unit"],
                "n_gpus": n, "steps": args.steps, "warmup": args.warmup,
-               "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+               "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+               "scaling": "strong" if args.shard == "heads" else "weak",
                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-               "config": {**head["config"], "parallelism": f"replicas x{n}" if n > 1 else "1 GPU"},
+               "config": {**head["config"],
+                          "parallelism": "1 GPU" if n == 1 else
+                          (f"KV-head shards x{n}" if args.shard == "heads" else f"replicas x{n}")},
                "roofline": head["roofline"], "e2e": head["e2e"],
                "gpu_launches": head["gpu_launches"], "clocks": clk,
                "device_planned_graph": head["device_planned_graph"],

@@ -33,7 +33,7 @@ from __future__ import annotations
 
 import math
 from dataclasses import dataclass, field
-from typing import Optional, Sequence
+from typing import Optional, Sequence, Tuple
 
 import numpy as np
 import torch
@@ -143,16 +143,29 @@ WORKLOADS = {
 
 
 def make_workload(name: str, device="cpu", causal: Optional[bool] = None, poison: bool = True,
-                  logical: Optional[bool] = None, max_seqs: Optional[int] = None) -> Problem:
+                  logical: Optional[bool] = None, max_seqs: Optional[int] = None,
+                  head_shard: Optional[Tuple[int, int]] = None) -> Problem:
     """One of the named workloads (see the module docstring).  ``max_seqs``
-    keeps only the first sequences (smaller cases for profiler captures)."""
+    keeps only the first sequences (smaller cases for profiler captures).
+    ``head_shard = (rank, n)``: rank's share of a KV-head split over n GPUs:
+    the same sequences and lengths, Hkv / n KV heads with their Hq / n query
+    heads (heads never interact, so the shards need no exchange); values are
+    drawn with a rank-specific seed."""
     dtype, hq, hkv, d, p, causal_default, vscale, seed, pool = WORKLOADS[name]
+    if head_shard is not None:
+        rank, n = head_shard
+        if n < 1 or hkv % n != 0 or not 0 <= rank < n:
+            raise ValueError(f"{name}: {hkv} KV heads do not split over {n} GPUs")
+        hq, hkv = hq // n, hkv // n
     gen = torch.Generator().manual_seed(seed)
     q_lens, kv_lens = _lengths(name, gen)
     if max_seqs is not None:
         q_lens, kv_lens = q_lens[:max_seqs], kv_lens[:max_seqs]
     if logical is None:
         logical = name == "tiny_mixed_f32"
+    if head_shard is not None and head_shard[0] > 0:
+        seed = seed + 7919 * head_shard[0]   # the lengths above are shared; pages and values per shard
+        gen.manual_seed(seed)
     return make_problem(q_lens, kv_lens, num_q_heads=hq, num_kv_heads=hkv, head_dim=d,
                         page_size=p, dtype=dtype, causal=causal_default if causal is None else causal,
                         seed=seed, pool=pool, value_scale=vscale, device=device, poison=poison,

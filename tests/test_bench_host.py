@@ -107,3 +107,31 @@ def test_roofline_uses_the_dominant_kernel():
     assert r["kernel"] == "prefill" and r["bound"] == "tensor"
     assert r["achieved"] == pytest.approx(1000.0)
     assert r["kernel_share"]["prefill"] == pytest.approx(1.0 / 1.2, abs=1e-4)
+
+
+def test_head_shards_split_heads_not_sequences():
+    """--shard heads: each rank gets the same sequences with Hkv / n KV heads
+    and their query heads; n must divide Hkv."""
+    full = I.make_workload("tiny_mixed_f32", device="cpu")
+    shards = [I.make_workload("mixed_96d_4c", device="cpu", poison=False, head_shard=(r, 4), max_seqs=6)
+              for r in range(4)]
+    ref = I.make_workload("mixed_96d_4c", device="cpu", poison=False, max_seqs=6)
+    for sh in shards:
+        assert list(sh.q_lens) == list(ref.q_lens) and list(sh.kv_lens) == list(ref.kv_lens)
+        assert sh.q.shape == (ref.q.shape[0], ref.q.shape[1] // 4, ref.q.shape[2])
+        assert sh.k_cache.shape[2] == ref.k_cache.shape[2] // 4
+    assert not torch.equal(shards[0].q, shards[1].q)          # rank-specific values
+    with pytest.raises(ValueError):
+        I.make_workload("tiny_mixed_f32", device="cpu", head_shard=(0, 2))   # 1 KV head
+    assert full.q.shape[1] == 4
+
+
+def test_head_shard_job_value():
+    """Value of a head-sharded job: bytes / FLOPs are summed over the ranks,
+    the batch's tokens are counted once."""
+    work = {"bytes": 10 ** 9, "flops": 10 ** 12, "tokens": 1000}
+    w = bench.rank_work(work, 4, "heads")
+    assert bench.value_of("mixed_96d_4c", w, 1.0, 4) == pytest.approx(1000 / 1e-3)
+    assert bench.value_of("decode_128", w, 1.0, 4) == pytest.approx(4 * 1e9 / 1e-3 / 1e9)
+    assert bench.rank_work(work, 4, "replicas") is work
+    assert bench.value_of("mixed_96d_4c", work, 1.0, 4) == pytest.approx(4 * 1000 / 1e-3)
