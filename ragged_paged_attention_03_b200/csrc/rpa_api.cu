@@ -130,8 +130,6 @@ struct HostPlan {
   int32_t n_partials = 0;
   int32_t decode_max_splits = 0;
   int32_t num_decode = 0, num_prefill = 0, num_generic = 0, num_empty = 0;
-  double decode_bytes = 0.0;     // K/V bytes the decode kernel streams
-  double prefill_flops = 0.0;    // visible (q, k) pairs x 4 D Hq
   int64_t prefill_ctx_tokens = 0, prefill_new_tokens = 0;
   PlanLayout layout{};
 };
@@ -163,7 +161,6 @@ void build_plan(const int32_t *cu, const int32_t *kv, int32_t n, const int32_t *
       }
       case kDecode: {
         ++hp.num_decode;
-        hp.decode_bytes += (double)kvl * d->num_kv_heads * d->head_dim * 4.0;
         const int32_t nblk = (kvl + kDecodeBlock - 1) / kDecodeBlock;
         if (nblk <= pack && nblk <= chunk) {
           // short: the whole sequence as one item of a packed CTA
@@ -207,12 +204,8 @@ void build_plan(const int32_t *cu, const int32_t *kv, int32_t n, const int32_t *
       }
       case kPrefill: {
         ++hp.num_prefill;
-        {
-          const double q = ql, c = (double)kvl - ql;
-          hp.prefill_flops += 4.0 * d->head_dim * d->num_q_heads * q * (c + (q + 1) / 2.0);
-          hp.prefill_ctx_tokens += (int64_t)kvl - ql;
-          hp.prefill_new_tokens += ql;
-        }
+        hp.prefill_ctx_tokens += (int64_t)kvl - ql;
+        hp.prefill_new_tokens += ql;
         const int32_t item_rows = prefill_item_rows(d->head_dim);
         for (int32_t r = 0; r < ql; r += item_rows) {
           PrefillTile t{};

@@ -203,7 +203,8 @@ def test_bad_device_lengths_write_nothing(oracle_mod):
     assert same_bits(slots.k_cache.cpu(), pre_k)
 
 
-FULL = [("decode_128", True), ("mixed_96d_4c", True), ("prefill_8x2048", True), ("prefill_8x2048", False)]
+FULL = [("decode_128", True), ("mixed_96d_4c", True), ("prefill_8x2048", True), ("prefill_8x2048", False),
+        ("long_d256", True)]
 
 
 @pytest.mark.parametrize("name,causal", FULL, ids=[f"{n}-{c}" for n, c in FULL])
