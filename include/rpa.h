@@ -255,7 +255,8 @@ RPA_API int rpa_profile_read(double *ms, int64_t *launches);
  * of 16 MiB that every GPU loading this part of the library holds until the
  * process exits.  A batch whose work items, combine rows or partial results
  * do not fit is rejected with RPA_ERR_SCRATCH_LIMIT before any device work
- * (about 8192 work items of 1024 tokens; partial results of
+ * (8192 work items of at most RPA_OPT_DECODE_CHUNK_BLOCKS 16-token blocks,
+ * 192 by default; partial results of
  * num_kv_heads * G * (head_dim + 1) floats per split item within ~15.6 MiB).
  * No cudaMalloc, cudaFree, cudaMallocHost or other allocating routine is
  * called.  The first call on a device looks up the array's device address

@@ -21,8 +21,10 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 
+#include "host_common.h"
 #include "kernels.h"
 #include "plan.h"
 #include "rpa.h"
@@ -39,7 +41,6 @@ constexpr int64_t kItemsOff = 256;
 constexpr int64_t kCombineOff = kItemsOff + kMaxItems * (int64_t)sizeof(DecodeItem);
 constexpr int64_t kPartialOff = kCombineOff + kMaxCombine * (int64_t)sizeof(CombineItem);
 constexpr int64_t kPartialFloats = (kScratchBytes - kPartialOff) / 4;
-constexpr int kChunkBlocks = 64;          // 16-token blocks per work item
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
@@ -87,10 +88,12 @@ extern "C" RPA_API int rpa_decode_noalloc(const void *q, const void *k_new, cons
   // ---- sizes against the fixed scratch (before touching any device)
   const int G = dims->num_q_heads / dims->num_kv_heads;
   const int64_t per_partial = (int64_t)dims->num_kv_heads * G * (D + 1);
+  // 16-token blocks per work item: rpa_forward's (RPA_OPT_DECODE_CHUNK_BLOCKS)
+  const int64_t chunk = decode_chunk_blocks();
   int64_t n_items = 0, n_partials = 0, n_combine = 0;
   for (int32_t s = 0; s < num_seqs; ++s) {
     const int64_t nblk = (kv_lens[s] + 15) / 16;
-    const int64_t nsplit = (nblk + kChunkBlocks - 1) / kChunkBlocks;
+    const int64_t nsplit = (nblk + chunk - 1) / chunk;
     n_items += nsplit;
     if (nsplit > 1) {
       n_partials += nsplit;
@@ -112,12 +115,12 @@ extern "C" RPA_API int rpa_decode_noalloc(const void *q, const void *k_new, cons
   }
   unsigned char *scratch = static_cast<unsigned char *>(g_scratch_ptr[dev]);
 
-  // ---- plan: near-equal chunks of at most kChunkBlocks 16-token blocks per sequence
+  // ---- plan: near-equal chunks of at most `chunk` 16-token blocks per sequence
   int32_t ni = 0, nc = 0, np = 0;
   for (int32_t s = 0; s < num_seqs; ++s) {
     const int32_t kvl = kv_lens[s];
     const int32_t nblk = (kvl + 15) / 16;
-    const int32_t nsplit = (nblk + kChunkBlocks - 1) / kChunkBlocks;
+    const int32_t nsplit = (int32_t)((nblk + chunk - 1) / chunk);
     const int32_t per = (nblk + nsplit - 1) / nsplit;
     const int32_t first = np;
     int32_t made = 0;
@@ -142,6 +145,11 @@ extern "C" RPA_API int rpa_decode_noalloc(const void *q, const void *k_new, cons
     }
   }
 
+  // longest items first (the kernel takes items in grid order, so the short
+  // ones fill the last wave); std::sort works in place and allocates nothing
+  std::sort(g_items, g_items + ni, [](const DecodeItem &x, const DecodeItem &y) {
+    return x.blk_end - x.blk_begin > y.blk_end - y.blk_begin;
+  });
   uint32_t *err = dev_flags ? dev_flags : reinterpret_cast<uint32_t *>(scratch);
   DecodeItem *d_items = reinterpret_cast<DecodeItem *>(scratch + kItemsOff);
   CombineItem *d_combine = reinterpret_cast<CombineItem *>(scratch + kCombineOff);

@@ -546,9 +546,7 @@ cudaError_t launch_prefill_t(const Problem &pb, const PrefillTile *tiles, int n_
 cudaError_t launch_prefill(const Problem &pb, const PrefillTile *tiles, int n_tiles, cudaStream_t stream) {
   if (n_tiles <= 0) return cudaSuccess;
   switch (pb.d) {
-    case 64: return launch_prefill_t<64>(pb, tiles, n_tiles, stream);
-    case 128: return launch_prefill_t<128>(pb, tiles, n_tiles, stream);
-    case 256: return launch_prefill_t<256>(pb, tiles, n_tiles, stream);
+    case 256: return launch_prefill_t<256>(pb, tiles, n_tiles, stream);   // 64 / 128: prefill2
     default: return cudaErrorInvalidValue;
   }
 }
