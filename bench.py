@@ -272,27 +272,22 @@ def host_call_us(prob, calls, stream):
 
 
 def time_e2e(prob, steps, warmup, flush, stream):
-    """Host buffers in, host buffers out: each step copies this step's Q, new
-    K/V and page table from pinned host memory, runs rpa_forward and copies
-    out and lse back, all inside the timed region."""
+    """Host buffers in, host buffers out, through rpa_forward_host: each step
+    copies this step's Q, new K/V and page table from pinned host memory,
+    runs the attention pass and copies out and lse back (the library overlaps
+    the copies with the kernels, group by group), all inside the timed
+    region.  The caches stay resident on the device."""
     from ragged_paged_attention_03_b200 import binding
     h = {k: getattr(prob, k).cpu().pin_memory() for k in ("q", "k_new", "v_new", "page_table")}
-    d = {k: torch.empty_like(getattr(prob, k)) for k in h}
-    out = torch.empty_like(prob.q)
-    lse = torch.empty(prob.q.shape[0], prob.num_q_heads, dtype=torch.float32, device=prob.q.device)
-    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h_out = torch.empty(prob.q.shape, dtype=prob.q.dtype).pin_memory()
+    h_lse = torch.empty(prob.q.shape[0], prob.num_q_heads, dtype=torch.float32).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in h.values())
     d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * 4
 
     def call():
-        for k in h:
-            d[k].copy_(h[k], non_blocking=True)
-        binding.rpa_forward(d["q"], d["k_new"], d["v_new"], prob.k_cache, prob.v_cache,
-                            d["page_table"], prob.cu_q_lens, prob.kv_lens, prob.distribution,
-                            prob.scale, prob.causal, out, lse, stream=stream)
-        h_out.copy_(out, non_blocking=True)
-        h_lse.copy_(lse, non_blocking=True)
+        binding.rpa_forward_host(h["q"], h["k_new"], h["v_new"], prob.k_cache, prob.v_cache, h["page_table"],
+                                 prob.cu_q_lens, prob.kv_lens, prob.distribution, prob.scale, prob.causal,
+                                 h_out, h_lse, stream=stream)
 
     with torch.cuda.stream(stream):
         for _ in range(warmup):

@@ -334,6 +334,72 @@ RPA_API int rpa_forward_device(const void *q, const void *k_new,
                                void *workspace, int64_t workspace_bytes,
                                uint32_t *dev_flags, void *stream);
 
+/*
+ * rpa_forward_host -- rpa_forward for a caller whose inputs and results are
+ * in host memory: q, k_new, v_new, page_table, out and lse are HOST pointers
+ * (same shapes and layouts as in rpa_forward); k_cache and v_cache stay
+ * DEVICE buffers (the cache is resident on the GPU).  cu_q_lens, kv_lens and
+ * distribution are host arrays as in rpa_forward.
+ *
+ * The operation is rpa_forward's (the same passages define it); the pages
+ * run it on device-resident data and say nothing of host buffers.  The call
+ * copies the new tokens in, runs the attention pass and copies out and lse
+ * back, queued on `stream` and the library's own streams, and returns
+ * without waiting: the host results are complete once `stream` has reached
+ * the end of the call (e.g. after cudaStreamSynchronize(stream)).  The host
+ * inputs must not be modified, nor the results read, before then.
+ * Page-locked host memory (cudaMallocHost or cudaHostRegister) lets the
+ * copies run asynchronously and overlap the kernels; with pageable memory
+ * the results are the same, the copies do not overlap and the call may
+ * return only after some of them have finished.
+ *
+ * Overlap: the batch is cut into at most RPA_HOST_MAX_GROUPS groups of whole
+ * consecutive sequences (rpa_host_groups gives the cut; batches with under
+ * 8 MiB of copies are one group, which runs entirely on `stream`).  With
+ * several groups, one library copy stream takes the page table and the
+ * first group's inputs, then all groups' plans, then the other groups'
+ * inputs; each group's kernels start once its own inputs have arrived
+ * (groups of decode sequences only on `stream`, the others on a library
+ * stream of the highest priority, so they may run concurrently), and its
+ * results go back on a library copy stream as soon as it is done.  The call
+ * joins every library stream back into `stream` before it returns.
+ *
+ * Results: the cache update is bit-identical to rpa_forward's; out and lse
+ * are those of rpa_forward run on each group (the same exact attention; the
+ * decode split-KV work split, and therefore the fp32 rounding order, can
+ * differ from one call over the whole batch).
+ *
+ * Workspace: per device, device staging for a call's inputs, results,
+ * plans and split-KV partials, and two pinned plan buffers (all grown on
+ * demand, kept until the process exits), plus rpa_forward's error word.
+ * Successive calls are ordered on the device against each other even on
+ * different streams.  Returns RPA_OK or an RPA_ERR_* code; all validation
+ * (rpa_forward's, over the whole batch) happens before anything is queued.
+ * RPA_ERR_CUDA / RPA_ERR_OOM after that point leave earlier groups' results
+ * possibly written.
+ */
+#define RPA_HOST_MAX_GROUPS 32
+RPA_API int rpa_forward_host(const void *q, const void *k_new,
+                             const void *v_new, void *k_cache, void *v_cache,
+                             const int32_t *page_table,
+                             const int32_t *cu_q_lens, const int32_t *kv_lens,
+                             int32_t num_seqs, const int32_t *distribution,
+                             float scale, int32_t causal, void *out,
+                             float *lse, const rpa_dims *dims, void *stream);
+
+/*
+ * rpa_host_groups -- the sequence groups rpa_forward_host would use for this
+ * batch: *num_groups groups, group g holding sequences [bounds[g],
+ * bounds[g+1]), bounds[0] = 0, bounds[*num_groups] = num_seqs.  bounds must
+ * hold RPA_HOST_MAX_GROUPS + 1 entries.  with_lse != 0 counts lse in the
+ * copy sizes (as a non-NULL lse does).  Host only; RPA_OK, or the RPA_ERR_*
+ * code of bad dims or cu_q_lens (not starting at 0, decreasing, or not
+ * ending at total_q_tokens).  num_seqs == 0 gives 0 groups.
+ */
+RPA_API int rpa_host_groups(const int32_t *cu_q_lens, int32_t num_seqs,
+                            const rpa_dims *dims, int32_t with_lse,
+                            int32_t *bounds, int32_t *num_groups);
+
 #ifdef __cplusplus
 }
 #endif

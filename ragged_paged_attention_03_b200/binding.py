@@ -262,3 +262,60 @@ def rpa_forward_device(q, k_new, v_new, k_cache, v_cache, page_table, cu_q_lens,
                                  workspace.numel(), _dev(dev_flags, "dev_flags", torch.int32), sptr)
     if rc != RPA_OK:
         raise RpaError(rc, "rpa_forward_device")
+
+
+RPA_HOST_MAX_GROUPS = 32
+_lib.rpa_forward_host.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _i32, _P, ctypes.c_float, _i32, _P, _P,
+                                  ctypes.POINTER(rpa_dims), _P]
+_lib.rpa_forward_host.restype = ctypes.c_int
+_lib.rpa_host_groups.argtypes = [_P, _i32, ctypes.POINTER(rpa_dims), _i32, _P, ctypes.POINTER(ctypes.c_int32)]
+_lib.rpa_host_groups.restype = ctypes.c_int
+
+
+def _host(t: Optional[torch.Tensor], name: str, dtype=None):
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def rpa_forward_host(q, k_new, v_new, k_cache, v_cache, page_table, cu_q_lens, kv_lens, distribution,
+                     scale: float, causal: bool, out, lse=None, stream=None) -> None:
+    """Calls rpa_forward_host: q, k_new, v_new, page_table, out and lse are
+    host (CPU, preferably pinned) tensors; k_cache / v_cache are CUDA tensors.
+    Asynchronous on `stream` (default: the current stream of the caches'
+    device): synchronise it before reading out / lse."""
+    dt = q.dtype
+    for name, t in (("k_new", k_new), ("v_new", v_new), ("k_cache", k_cache),
+                    ("v_cache", v_cache), ("out", out)):
+        if t.dtype != dt:
+            raise TypeError(f"{name} dtype {t.dtype} != q dtype {dt}")
+    cu, kv, dist = _host_i32(cu_q_lens), _host_i32(kv_lens), _host_i32(distribution)
+    dims = make_dims(q, k_cache, page_table)
+    if stream is None:
+        stream = torch.cuda.current_stream(k_cache.device)
+    sptr = ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+    rc = _lib.rpa_forward_host(_host(q, "q"), _host(k_new, "k_new"), _host(v_new, "v_new"),
+                               _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                               _host(page_table, "page_table", torch.int32), _hp(cu), _hp(kv), len(kv),
+                               _hp(dist), float(scale), int(bool(causal)), _host(out, "out"),
+                               _host(lse, "lse", torch.float32), ctypes.byref(dims), sptr)
+    if rc != RPA_OK:
+        raise RpaError(rc, "rpa_forward_host")
+
+
+def rpa_host_groups(cu_q_lens, dims: rpa_dims, with_lse: bool = True) -> np.ndarray:
+    """Sequence group boundaries rpa_forward_host uses for this batch."""
+    cu = _host_i32(cu_q_lens)
+    bounds = np.zeros(RPA_HOST_MAX_GROUPS + 1, dtype=np.int32)
+    n = ctypes.c_int32(0)
+    rc = _lib.rpa_host_groups(_hp(cu), len(cu) - 1, ctypes.byref(dims), int(bool(with_lse)), _hp(bounds),
+                              ctypes.byref(n))
+    if rc != RPA_OK:
+        raise RpaError(rc, "rpa_host_groups")
+    return bounds[:n.value + 1].copy()

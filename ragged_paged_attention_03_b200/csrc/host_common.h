@@ -1,5 +1,5 @@
 // host_common.h -- host-side helpers shared by the entry points of the
-// library (rpa_api.cu, device_plan.cu): geometry validation and the
+// library (rpa_api.cu, device_plan.cu, host_io.cu): validation and the
 // effective values of the process-wide planner options.
 #pragma once
 #include <stdint.h>
@@ -10,6 +10,10 @@ namespace rpa {
 
 // RPA_OK, or the RPA_ERR_* code rpa_forward returns for these dims.
 int validate_dims(const rpa_dims *d);
+// ... for these host lengths (cu_q_lens [n+1], kv_lens [n]) under dims d.
+int validate_lengths(const int32_t *cu, const int32_t *kv, int32_t n, const rpa_dims *d);
+// ... for this distribution (NULL is always valid) of valid lengths.
+int validate_distribution(const int32_t *dist, const int32_t *cu, const int32_t *kv, int32_t n);
 
 // Effective planner options (defaults and clamps applied).
 int64_t decode_chunk_blocks();   // 16-token blocks per decode work item

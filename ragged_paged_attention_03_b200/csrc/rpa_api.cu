@@ -20,6 +20,7 @@
 
 #include "host_common.h"
 #include "kernels.h"
+#include "forward_internal.h"
 #include "plan.h"
 #include "rpa.h"
 
@@ -77,8 +78,6 @@ int validate_dims(const rpa_dims *d) {
   return RPA_OK;
 }
 
-namespace {
-
 int validate_lengths(const int32_t *cu, const int32_t *kv, int32_t n, const rpa_dims *d) {
   if (n < 0) return RPA_ERR_INVALID_ARG;
   if (n == 0) return d->total_q_tokens == 0 ? RPA_OK : RPA_ERR_LENGTHS;
@@ -105,6 +104,8 @@ int validate_distribution(const int32_t *dist, const int32_t *cu, const int32_t 
   return RPA_OK;
 }
 
+namespace {
+
 enum Route { kEmpty, kGeneric, kDecode, kPrefill };
 
 // Kernel choice for one sequence.  With a distribution the ranges decide the
@@ -120,19 +121,7 @@ Route route_of(int32_t ql, int32_t kvl, int dtype, int cls) {
   return kPrefill;
 }
 
-struct HostPlan {
-  std::vector<GenericSeq> generic;
-  std::vector<DecodeItem> decode;
-  std::vector<DecodeItem> decode_packed;   // whole short sequences, four per CTA
-  std::vector<CombineItem> combine;
-  std::vector<PrefillTile> prefill;
-  int32_t n_generic_rows = 0;
-  int32_t n_partials = 0;
-  int32_t decode_max_splits = 0;
-  int32_t num_decode = 0, num_prefill = 0, num_generic = 0, num_empty = 0;
-  int64_t prefill_ctx_tokens = 0, prefill_new_tokens = 0;
-  PlanLayout layout{};
-};
+}  // namespace
 
 void build_plan(const int32_t *cu, const int32_t *kv, int32_t n, const int32_t *dist,
                 const rpa_dims *d, HostPlan &hp) {
@@ -277,6 +266,8 @@ void serialize(const HostPlan &hp, int32_t *dst) {
     memcpy(dst + L.prefill_off, hp.prefill.data(), hp.prefill.size() * sizeof(PrefillTile));
 }
 
+namespace {
+
 // ---------------------------------------------------------------- workspace
 //
 // Per device: a ring of slots, each with a pinned host staging buffer, a
@@ -304,6 +295,7 @@ struct DeviceWs {
   bool init = false;
   uint32_t *err = nullptr;
   cudaStream_t side = nullptr;  // prefill of mixed batches runs here
+  cudaEvent_t fork = nullptr, join = nullptr;   // side-stream order for launch_planned
   int sms = 0;
   Slot slots[kSlots];
   int next = 0;
@@ -315,6 +307,9 @@ int ensure_init(DeviceWs &ws) {
   if (ws.init) return RPA_OK;
   if (cudaMalloc(&ws.err, sizeof(uint32_t)) != cudaSuccess) return RPA_ERR_OOM;
   if (cudaMemset(ws.err, 0, sizeof(uint32_t)) != cudaSuccess) return RPA_ERR_CUDA;
+  if (cudaEventCreateWithFlags(&ws.fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&ws.join, cudaEventDisableTiming) != cudaSuccess)
+    return RPA_ERR_CUDA;
   for (auto &s : ws.slots)
     if (cudaEventCreateWithFlags(&s.done, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming) != cudaSuccess ||
@@ -410,7 +405,115 @@ cudaError_t traced(int kind, cudaStream_t stream, F &&launch) {
   return e;
 }
 
+
+// The kernels of one planned call, queued on `stream` (the caller holds
+// ws.mu).  A batch with both prefill and decode work runs them
+// concurrently: the compute-bound prefill kernel on the high-priority side
+// stream, queued first, takes the SMs (one whole-SM CTA each); the
+// bandwidth-bound decode kernel on the caller's stream fills every SM its
+// prefill CTA leaves, so the prefill's uneven finish is covered instead of
+// waited for.  fork / join order the side stream against `stream`.
+cudaError_t launch_kernels(DeviceWs &ws, const HostPlan &hp, const int32_t *dev_plan, float *partials,
+                           Problem pb, cudaStream_t stream, cudaEvent_t fork, cudaEvent_t join) {
+  pb.err = ws.err;
+  const PlanLayout &L = hp.layout;
+  const int G = pb.hq / pb.hkv;
+  float *partial_o = partials;
+  float *partial_lse = partials ? partials + L.n_partials * pb.hkv * G * pb.d : nullptr;
+  cudaError_t e = cudaSuccess;
+  const bool mixed = L.n_prefill_tiles > 0 &&
+                     (L.n_decode_items > 0 || L.n_decode_packed > 0 || L.n_generic_rows > 0) &&
+                     g_opt_concurrent_mixed.load() >= 0;
+  cudaStream_t pstream = stream;
+  int prefill_ctas = 0;
+  if (mixed) {
+    const int64_t k = g_opt_prefill_sms.load();
+    prefill_ctas = k > 0 ? (int)std::min<int64_t>(k, ws.sms) : 0;   // 0: one per SM
+    pstream = ws.side;
+    if (cudaEventRecord(fork, stream) != cudaSuccess || cudaStreamWaitEvent(pstream, fork, 0) != cudaSuccess)
+      return cudaErrorUnknown;
+  }
+  if (L.n_prefill_tiles > 0 && e == cudaSuccess)
+    e = traced(RPA_KERNEL_PREFILL, pstream, [&] {
+      const PrefillTile *tiles = (const PrefillTile *)(dev_plan + L.prefill_off);
+      // context-heavy prefill (chunked rows after a long cache) gathers
+      // latency-bound paged blocks and writes few new rows: a producer warp
+      // per operand; fresh prefill keeps two warps for the cache update
+      const int64_t lo = g_opt_prefill_loaders.load();
+      const bool split = lo == 2 || (lo != 1 && hp.prefill_ctx_tokens > hp.prefill_new_tokens);
+      return pb.d <= 128 ? launch_prefill2(pb, tiles, (int)L.n_prefill_tiles, prefill_ctas, split, pstream)
+                         : launch_prefill(pb, tiles, (int)L.n_prefill_tiles, pstream);
+    });
+  if (mixed && cudaEventRecord(join, pstream) != cudaSuccess) e = cudaErrorUnknown;
+  if (L.n_decode_items > 0 && e == cudaSuccess)
+    e = traced(RPA_KERNEL_DECODE, stream, [&] {
+      return launch_decode(pb, (const DecodeItem *)(dev_plan + L.decode_off), (int)L.n_decode_items, partial_o,
+                           partial_lse, false, stream);
+    });
+  if (L.n_decode_packed > 0 && e == cudaSuccess)
+    e = traced(RPA_KERNEL_DECODE, stream, [&] {
+      return launch_decode(pb, (const DecodeItem *)(dev_plan + L.decode_packed_off), (int)L.n_decode_packed,
+                           partial_o, partial_lse, true, stream);
+    });
+  if (L.n_combine > 0 && e == cudaSuccess)
+    e = traced(RPA_KERNEL_COMBINE, stream, [&] {
+      return launch_combine(pb, (const CombineItem *)(dev_plan + L.combine_off), (int)L.n_combine, partial_o,
+                            partial_lse, stream);
+    });
+  if (L.n_generic_rows > 0 && e == cudaSuccess)
+    e = traced(RPA_KERNEL_GENERIC, stream, [&] {
+      return launch_generic(pb, (const GenericSeq *)(dev_plan + L.generic_off), (int)L.n_generic_seqs,
+                            (int)L.n_generic_rows, stream);
+    });
+  // join: the caller's stream waits for the side stream (also on errors,
+  // so that nothing of this call is left running unordered)
+  if (mixed && cudaStreamWaitEvent(stream, join, 0) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;
+  return e;
+}
+
 }  // namespace
+
+int64_t plan_partial_floats(const HostPlan &hp, const rpa_dims &d) {
+  return hp.layout.n_partials * (int64_t)d.num_q_heads * (d.head_dim + 1);
+}
+
+Problem problem_of(const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                   const int32_t *page_table, void *out, float *lse, const rpa_dims &d, float scale,
+                   int32_t causal) {
+  Problem pb{};
+  pb.q = q;
+  pb.k_new = k_new;
+  pb.v_new = v_new;
+  pb.k_cache = k_cache;
+  pb.v_cache = v_cache;
+  pb.page_table = page_table;
+  pb.out = out;
+  pb.lse = lse;
+  pb.hq = d.num_q_heads;
+  pb.hkv = d.num_kv_heads;
+  pb.d = d.head_dim;
+  pb.p = d.page_size;
+  pb.num_pages = d.num_pages;
+  pb.max_pages = d.max_pages_per_seq;
+  pb.dtype = d.dtype;
+  pb.causal = causal ? 1 : 0;
+  pb.scale = scale;
+  pb.total_q = d.total_q_tokens;
+  return pb;
+}
+
+int launch_planned(const HostPlan &hp, const int32_t *dev_plan, float *partials, Problem pb,
+                   cudaStream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RPA_ERR_CUDA;
+  DeviceWs &ws = g_ws[dev];
+  std::lock_guard<std::mutex> lock(ws.mu);
+  const int rc = ensure_init(ws);
+  if (rc) return rc;
+  return launch_kernels(ws, hp, dev_plan, partials, pb, stream, ws.fork, ws.join) == cudaSuccess ? RPA_OK
+                                                                                                  : RPA_ERR_CUDA;
+}
+
 }  // namespace rpa
 
 using namespace rpa;
@@ -492,93 +595,15 @@ extern "C" RPA_API int rpa_forward(const void *q, const void *k_new, const void 
     Slot &slot = ws.slots[ws.next];
     ws.next = (ws.next + 1) % kSlots;
 
-    const int G = dims->num_q_heads / dims->num_kv_heads;
-    const int64_t per_partial = (int64_t)dims->num_kv_heads * G * (dims->head_dim + 1);
-    rc = grow_slot(slot, hp.layout.total_words, hp.layout.n_partials * per_partial);
+    rc = grow_slot(slot, hp.layout.total_words, plan_partial_floats(hp, *dims));
     if (rc) return rc;
     serialize(hp, slot.host);
     if (hp.layout.total_words > 0 &&
         cudaMemcpyAsync(slot.dev, slot.host, hp.layout.total_words * sizeof(int32_t),
                         cudaMemcpyHostToDevice, stream) != cudaSuccess)
       return RPA_ERR_CUDA;
-
-    Problem pb{};
-    pb.q = q;
-    pb.k_new = k_new;
-    pb.v_new = v_new;
-    pb.k_cache = k_cache;
-    pb.v_cache = v_cache;
-    pb.page_table = page_table;
-    pb.out = out;
-    pb.lse = lse;
-    pb.err = ws.err;
-    pb.hq = dims->num_q_heads;
-    pb.hkv = dims->num_kv_heads;
-    pb.d = dims->head_dim;
-    pb.p = dims->page_size;
-    pb.num_pages = dims->num_pages;
-    pb.max_pages = dims->max_pages_per_seq;
-    pb.dtype = dims->dtype;
-    pb.causal = causal ? 1 : 0;
-    pb.scale = scale;
-    pb.total_q = T;
-
-    const PlanLayout &L = hp.layout;
-    float *partial_o = slot.partial;
-    float *partial_lse = slot.partial ? slot.partial + L.n_partials * dims->num_kv_heads * G * dims->head_dim : nullptr;
-    cudaError_t e = cudaSuccess;
-    // A batch with both prefill and decode work runs them concurrently: the
-    // compute-bound prefill kernel on the high-priority side stream, queued
-    // first, takes the SMs (one whole-SM CTA each); the bandwidth-bound decode
-    // kernel on the caller's stream fills every SM its prefill CTA leaves, so
-    // the prefill's uneven finish is covered instead of waited for.
-    const bool mixed = L.n_prefill_tiles > 0 &&
-                       (L.n_decode_items > 0 || L.n_decode_packed > 0 || L.n_generic_rows > 0) &&
-                       g_opt_concurrent_mixed.load() >= 0;
-    cudaStream_t pstream = stream;
-    int prefill_ctas = 0;
-    if (mixed) {
-      const int64_t k = g_opt_prefill_sms.load();
-      prefill_ctas = k > 0 ? (int)std::min<int64_t>(k, ws.sms) : 0;   // 0: one per SM
-      pstream = ws.side;
-      if (cudaEventRecord(slot.fork, stream) != cudaSuccess || cudaStreamWaitEvent(pstream, slot.fork, 0) != cudaSuccess)
-        return RPA_ERR_CUDA;
-    }
-    if (L.n_prefill_tiles > 0 && e == cudaSuccess)
-      e = traced(RPA_KERNEL_PREFILL, pstream, [&] {
-        const PrefillTile *tiles = (const PrefillTile *)(slot.dev + L.prefill_off);
-        // context-heavy prefill (chunked rows after a long cache) gathers
-        // latency-bound paged blocks and writes few new rows: a producer warp
-        // per operand; fresh prefill keeps two warps for the cache update
-        const int64_t lo = g_opt_prefill_loaders.load();
-        const bool split = lo == 2 || (lo != 1 && hp.prefill_ctx_tokens > hp.prefill_new_tokens);
-        return pb.d <= 128 ? launch_prefill2(pb, tiles, (int)L.n_prefill_tiles, prefill_ctas, split, pstream)
-                           : launch_prefill(pb, tiles, (int)L.n_prefill_tiles, pstream);
-      });
-    if (mixed && cudaEventRecord(slot.join, pstream) != cudaSuccess) e = cudaErrorUnknown;
-    if (L.n_decode_items > 0 && e == cudaSuccess)
-      e = traced(RPA_KERNEL_DECODE, stream, [&] {
-        return launch_decode(pb, (const DecodeItem *)(slot.dev + L.decode_off),
-                             (int)L.n_decode_items, partial_o, partial_lse, false, stream);
-      });
-    if (L.n_decode_packed > 0 && e == cudaSuccess)
-      e = traced(RPA_KERNEL_DECODE, stream, [&] {
-        return launch_decode(pb, (const DecodeItem *)(slot.dev + L.decode_packed_off),
-                             (int)L.n_decode_packed, partial_o, partial_lse, true, stream);
-      });
-    if (L.n_combine > 0 && e == cudaSuccess)
-      e = traced(RPA_KERNEL_COMBINE, stream, [&] {
-        return launch_combine(pb, (const CombineItem *)(slot.dev + L.combine_off),
-                              (int)L.n_combine, partial_o, partial_lse, stream);
-      });
-    if (L.n_generic_rows > 0 && e == cudaSuccess)
-      e = traced(RPA_KERNEL_GENERIC, stream, [&] {
-        return launch_generic(pb, (const GenericSeq *)(slot.dev + L.generic_off),
-                              (int)L.n_generic_seqs, (int)L.n_generic_rows, stream);
-      });
-    // join: the caller's stream waits for the side stream (also on errors,
-    // so that nothing of this call is left running unordered)
-    if (mixed && cudaStreamWaitEvent(stream, slot.join, 0) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;
+    Problem pb = problem_of(q, k_new, v_new, k_cache, v_cache, page_table, out, lse, *dims, scale, causal);
+    const cudaError_t e = launch_kernels(ws, hp, slot.dev, slot.partial, pb, stream, slot.fork, slot.join);
     if (cudaEventRecord(slot.done, stream) == cudaSuccess) slot.pending = true;
     return e == cudaSuccess ? RPA_OK : RPA_ERR_CUDA;
   } catch (const std::bad_alloc &) {

@@ -262,3 +262,55 @@ def test_forward_device_host_checks(rb):
     assert call(max_seqs=0) == 0                  # no sequence slot: nothing to do
     assert call(dd=dims(total_q_tokens=0)) == 0   # no token row: nothing to do
     assert rb.rpa_status_string(rb.RPA_ERR_WORKSPACE) == "workspace too small or misaligned"
+
+
+def test_host_groups(rb):
+    """The sequence groups rpa_forward_host pipelines: one group under 8 MiB
+    of copies, one per long sequence, a decode run kept apart from the long
+    sequences after it, in order, covering every sequence."""
+    assert list(rb.rpa_host_groups(np.arange(129), dims(total_q_tokens=128))) == [0, 128]
+    cu = np.arange(9) * 2048
+    assert list(rb.rpa_host_groups(cu, dims(total_q_tokens=16384))) == list(range(9))
+    cu = np.concatenate([np.arange(97), 96 + np.arange(1, 5) * 512])
+    assert list(rb.rpa_host_groups(cu, dims(total_q_tokens=int(cu[-1])))) == [0, 96, 97, 98, 99, 100]
+    cu = np.concatenate([[0], np.cumsum(np.random.default_rng(3).integers(0, 3000, 1000))])
+    b = rb.rpa_host_groups(cu, dims(total_q_tokens=int(cu[-1])))
+    assert 1 < len(b) - 1 <= rb.RPA_HOST_MAX_GROUPS and b[0] == 0 and b[-1] == 1000
+    assert (np.diff(b) > 0).all()
+    # 1000 tokens at 8/2 heads: ~5 MB of copies in bf16 (one group), twice
+    # that in fp32 (two); lse adds Hq floats per token
+    small, d8 = np.array([0, 500, 1000]), dict(total_q_tokens=1000, num_q_heads=8, num_kv_heads=2)
+    assert len(rb.rpa_host_groups(small, dims(**d8))) == 2
+    assert len(rb.rpa_host_groups(small, dims(dtype=0, **d8))) == 3
+    edge = np.array([0, 815, 1630])     # 8 MiB with lse, just under without
+    assert len(rb.rpa_host_groups(edge, dims(**dict(d8, total_q_tokens=1630)), True)) == 3
+    assert len(rb.rpa_host_groups(edge, dims(**dict(d8, total_q_tokens=1630)), False)) == 2
+    with pytest.raises(rb.RpaError) as e:
+        rb.rpa_host_groups(np.array([1, 2]), dims(total_q_tokens=2))
+    assert e.value.code == 3
+    with pytest.raises(rb.RpaError) as e:
+        rb.rpa_host_groups(np.array([0, 5, 4]), dims(total_q_tokens=4))
+    assert e.value.code == 3
+
+
+def test_forward_host_checks(rb):
+    """rpa_forward_host validates the whole batch on the host before any
+    device work, and without a usable device fails with RPA_ERR_CUDA."""
+    lib = rb.library()
+    fake = ctypes.c_void_p(0x1000)
+
+    def call(q_lens, kv_lens, scale=1.0, ptr=fake, dist=None):
+        cu = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+        kv = np.array(kv_lens, np.int32)
+        d = dims(total_q_tokens=int(cu[-1]))
+        dp = None if dist is None else np.array(dist, np.int32).ctypes.data_as(ctypes.c_void_p)
+        return lib.rpa_forward_host(ptr, fake, fake, fake, fake, fake, cu.ctypes.data_as(ctypes.c_void_p),
+                                    kv.ctypes.data_as(ctypes.c_void_p), len(kv_lens), dp, ctypes.c_float(scale),
+                                    1, fake, None, ctypes.byref(d), None)
+    assert call([2], [1]) == 3                    # kv_len < q_len
+    assert call([1], [4], scale=0.0) == 1
+    assert call([1], [4], ptr=None) == 1
+    assert call([1, 3], [4, 3], dist=[0, 2, 2]) == 4   # sequence 0 is not a fresh prefill
+    assert call([], []) == 0                      # empty batch: a no-op
+    if not torch.cuda.is_available():
+        assert call([1], [4]) == 6
