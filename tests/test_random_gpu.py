@@ -1,11 +1,13 @@
-"""Seeded random batches against the oracle, through both entry points.
+"""Seeded random batches against the oracle, through all three entry points.
 
 Each case draws a geometry (head_dim 64/128/256, G = Hq/Hkv from 1 to 8,
 page size 8..256, causal or not, bf16 or fp32) and a batch that mixes
 decode, fresh-prefill, chunked-prefill and empty sequences with lengths
-across block and page boundaries.  rpa_forward (host planner) and
-rpa_forward_device (planner kernel) must each match the oracle within the
-stated tolerances, with the cache bit-exact.
+across block and page boundaries.  rpa_forward (host planner),
+rpa_forward_device (planner kernel) and rpa_forward_host (host buffers,
+split into copy-overlapped groups when the batch's copies reach 8 MiB) must
+each match the oracle within the stated tolerances, with the cache
+bit-exact.
 """
 import numpy as np
 import pytest
@@ -15,6 +17,7 @@ from ragged_paged_attention_03_b200 import inputs as I
 
 from harness import check_close, f64, oracle_full, run_gpu, same_bits, to_device
 from test_device_plan_gpu import Slots, check_slots
+from test_host_io_gpu import run_host
 
 pytestmark = pytest.mark.gpu
 
@@ -76,3 +79,8 @@ def test_random_batch(oracle_mod, seed):
     slots.load(prob)
     slots.call()
     check_slots(oracle_mod, slots, prob)
+    # host buffers in and out
+    out_h, lse_h, kc_h, vc_h, flags = run_host(prob, use_distribution=False)
+    assert flags == 0, f"device error flags {flags:#x}"
+    check_close(f64(out_h), out_ref, f64(lse_h), lse_ref, prob.dtype, f"{prob.name} host {c}")
+    assert same_bits(kc_h, kc_ref) and same_bits(vc_h, vc_ref), f"{prob.name}: host-call cache differs"
