@@ -110,10 +110,20 @@ struct Unit {
   int rows_t[2], n_t[2];
 };
 
+// Tile descriptor of unit u, or an empty one (rows == 0) past the last
+// unit.  Each role loads the next unit's descriptor at the top of the
+// current unit, so that a unit change does not start with a dependent
+// global read of the plan.
+__device__ __forceinline__ PrefillTile load_tile(const PrefillTile *tiles, int u, int n_units, int hq) {
+  PrefillTile t{};
+  if (u < n_units) t = tiles[u / hq];
+  return t;
+}
+
 template <int BM, int BN>
-__device__ __forceinline__ Unit make_unit(const PrefillTile *tiles, int u, const Problem &pb) {
+__device__ __forceinline__ Unit make_unit(const PrefillTile &tile, int u, const Problem &pb) {
   Unit w;
-  w.tile = tiles[u / pb.hq];
+  w.tile = tile;
   w.h = u % pb.hq;
   w.hk = w.h / (pb.hq / pb.hkv);
   w.c = w.tile.kv_len - w.tile.q_len;
@@ -202,8 +212,10 @@ __device__ __forceinline__ void mma_loop(Bars2 *bars, volatile int *abort_flag, 
   uint32_t *err = pb.err;
   int g0 = 0, gt0 = 0, gt1 = 0, ep0 = 0, ep1 = 0, uq = 0;
   bool ok = true;
+  PrefillTile next = load_tile(tiles, unit_of(0), n_units, pb.hq);
   for (int r = 0, u = unit_of(0); ok && u < n_units; u = unit_of(++r), ++uq) {
-    const Unit w = make_unit<BM, BN>(tiles, u, pb);
+    const Unit w = make_unit<BM, BN>(next, u, pb);
+    next = load_tile(tiles, unit_of(r + 1), n_units, pb.hq);
     if (w.tile.rows == 0) break;   // end of a device-planned tile list
     const int n0 = w.n_t[0], n1 = w.n_t[1], nb = w.nb;
     ok = wait_all(&bars->q_full, (uint32_t)(uq & 1), abort_flag, err);
@@ -281,8 +293,10 @@ __device__ __forceinline__ void produce_kv(Bars2 *bars, volatile int *abort_flag
   bool fix_pending = false;
   int uq = 0;           // units started
   bool ok = true;
+  PrefillTile next = load_tile(tiles, unit_of(0), n_units, pb.hq);
   for (int r = 0, u = unit_of(0); ok && u < n_units; u = unit_of(++r), ++uq) {
-    const Unit w = make_unit<BM, BN>(tiles, u, pb);
+    const Unit w = make_unit<BM, BN>(next, u, pb);
+    next = load_tile(tiles, unit_of(r + 1), n_units, pb.hq);
     if (w.tile.rows == 0) break;   // end of a device-planned tile list
     const int32_t *pt_row = pb.page_table + (size_t)w.tile.seq * pb.max_pages;
     // Q of both tiles, once the previous unit's QK MMAs are done with sQ
@@ -435,8 +449,10 @@ __device__ __forceinline__ void produce(Bars2 *bars, volatile int *abort_flag, c
   bool fix_pending = false;
   int uq = 0;           // units started
   bool ok = true;
+  PrefillTile next = load_tile(tiles, unit_of(0), n_units, pb.hq);
   for (int r = 0, u = unit_of(0); ok && u < n_units; u = unit_of(++r), ++uq) {
-    const Unit w = make_unit<BM, BN>(tiles, u, pb);
+    const Unit w = make_unit<BM, BN>(next, u, pb);
+    next = load_tile(tiles, unit_of(r + 1), n_units, pb.hq);
     if (w.tile.rows == 0) break;   // end of a device-planned tile list
     const int32_t *pt_row = pb.page_table + (size_t)w.tile.seq * pb.max_pages;
     if (!IS_V) {
@@ -545,8 +561,10 @@ __device__ __forceinline__ void cache_update(const Problem pb, const PrefillTile
   const __nv_bfloat16 *vn = reinterpret_cast<const __nv_bfloat16 *>(pb.v_new);
   __nv_bfloat16 *kc = reinterpret_cast<__nv_bfloat16 *>(pb.k_cache);
   __nv_bfloat16 *vc = reinterpret_cast<__nv_bfloat16 *>(pb.v_cache);
+  PrefillTile next = load_tile(tiles, unit_of(0), n_units, pb.hq);
   for (int r = 0, u = unit_of(0); u < n_units; u = unit_of(++r)) {
-    const Unit w = make_unit<BM, BN>(tiles, u, pb);
+    const Unit w = make_unit<BM, BN>(next, u, pb);
+    next = load_tile(tiles, unit_of(r + 1), n_units, pb.hq);
     if (w.tile.rows == 0) break;   // end of a device-planned tile list
     const int32_t *pt_row = pb.page_table + (size_t)w.tile.seq * pb.max_pages;
     const int gidx = w.h % G;
@@ -673,8 +691,10 @@ __global__ void __launch_bounds__(384, 1)
     int gt = 0;                                  // blocks of this tile consumed so far
     int ep = 0;                                  // units in which this tile had rows
     bool ok = true;
+    PrefillTile next = load_tile(tiles, unit_of(0), n_units, pb.hq);
     for (int r = 0, u = unit_of(0); ok && u < n_units; u = unit_of(++r)) {
-      const Unit w = make_unit<BM, BN>(tiles, u, pb);
+      const Unit w = make_unit<BM, BN>(next, u, pb);
+      next = load_tile(tiles, unit_of(r + 1), n_units, pb.hq);
       if (w.tile.rows == 0) break;   // end of a device-planned tile list
       // tile-uniform selects keep the unit in registers (no local memory)
       const int n = t ? w.n_t[1] : w.n_t[0];
