@@ -166,3 +166,29 @@ def test_empty_and_zero_length_groups(oracle_mod):
     binding.rpa_forward_host(empty.q, empty.k_new, empty.v_new, kc, empty.v_cache.cuda(),
                              empty.page_table, empty.cu_q_lens, empty.kv_lens, None, empty.scale,
                              True, empty.q.clone(), None)
+
+
+def test_calls_on_two_streams(oracle_mod):
+    """Two pipelined calls queued back to back on different streams share
+    the library's staging buffers; the second must wait for the first, and
+    both results must be the oracle's."""
+    from ragged_paged_attention_03_b200 import binding
+    probs = [pipelined_problem(seed=80), pipelined_problem(seed=81, causal=False)]
+    refs = [oracle_full(oracle_mod, p) for p in probs]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    res = []
+    for prob, st in zip(probs, streams):
+        q, kn, vn, pt = (t.cpu().contiguous().pin_memory() for t in (prob.q, prob.k_new, prob.v_new, prob.page_table))
+        out = torch.full(prob.q.shape, float("nan"), dtype=prob.q.dtype).pin_memory()
+        lse = torch.full((prob.q.shape[0], prob.q.shape[1]), float("nan")).pin_memory()
+        kc, vc = prob.k_cache.cuda().clone(), prob.v_cache.cuda().clone()
+        torch.cuda.synchronize()
+        binding.rpa_forward_host(q, kn, vn, kc, vc, pt, prob.cu_q_lens, prob.kv_lens, prob.distribution,
+                                 prob.scale, prob.causal, out, lse, stream=st)
+        res.append((out, lse, kc, vc, (q, kn, vn, pt)))
+    for st in streams:
+        st.synchronize()
+    assert binding.rpa_device_status() == 0
+    for prob, (out_ref, lse_ref, kc_ref, vc_ref), (out, lse, kc, vc, _) in zip(probs, refs, res):
+        check_close(f64(out), out_ref, f64(lse), lse_ref, prob.dtype, prob.name + " two streams")
+        assert same_bits(kc, kc_ref) and same_bits(vc, vc_ref)
