@@ -200,7 +200,9 @@ enum {
                                       concurrently, prefill on a
                                       highest-priority library stream that the
                                       caller's stream joins before the call
-                                      returns; < 0: one after the other */
+                                      returns (rpa_forward_host: its groups
+                                      with prefill rows likewise); < 0: one
+                                      after the other */
   RPA_OPT_PREFILL_LOADERS = 5,     /* TMA producer warps of the head_dim <= 128
                                       prefill kernel: 1 (K and V share one), 2
                                       (one each; the cache update gets one warp

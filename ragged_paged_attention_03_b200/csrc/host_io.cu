@@ -343,8 +343,11 @@ extern "C" RPA_API int rpa_forward_host(const void *q, const void *k_new, const 
       const int32_t s0 = bounds[g];
       const int64_t t0 = cu_q_lens[s0], nt = cu_q_lens[bounds[g + 1]] - t0;
       if (nt == 0) continue;   // only q_len = 0 sequences: nothing to write or read back
-      cudaStream_t cs = one ? stream : has_prefill[g] ? io.comp_hi : stream;
-      cudaStream_t os = one ? stream : has_prefill[g] ? io.d2h_hi : io.d2h;
+      // RPA_OPT_CONCURRENT_MIXED < 0: every group's kernels in order on the
+      // caller's stream (as rpa_forward then runs prefill and decode serially)
+      const bool side = !one && has_prefill[g] && concurrent_mixed();
+      cudaStream_t cs = side ? io.comp_hi : stream;
+      cudaStream_t os = one ? stream : side ? io.d2h_hi : io.d2h;
       rpa_dims dg = *dims;
       dg.total_q_tokens = (int32_t)nt;
       if (!one) e = cudaStreamWaitEvent(cs, io.in[g], 0);
