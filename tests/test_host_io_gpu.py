@@ -192,3 +192,14 @@ def test_calls_on_two_streams(oracle_mod):
     for prob, (out_ref, lse_ref, kc_ref, vc_ref), (out, lse, kc, vc, _) in zip(probs, refs, res):
         check_close(f64(out), out_ref, f64(lse), lse_ref, prob.dtype, prob.name + " two streams")
         assert same_bits(kc, kc_ref) and same_bits(vc, vc_ref)
+
+
+def test_serial_groups_option(oracle_mod):
+    """RPA_OPT_CONCURRENT_MIXED < 0: every group in order on the caller's
+    stream; the results are the oracle's all the same."""
+    from ragged_paged_attention_03_b200 import binding
+    old = binding.rpa_set_option(binding.RPA_OPT_CONCURRENT_MIXED, -1)
+    try:
+        check_vs_oracle(oracle_mod, pipelined_problem(seed=90))
+    finally:
+        binding.rpa_set_option(binding.RPA_OPT_CONCURRENT_MIXED, old)
