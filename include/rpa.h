@@ -225,8 +225,11 @@ enum { RPA_KERNEL_GENERIC = 0, RPA_KERNEL_DECODE = 1, RPA_KERNEL_COMBINE = 2,
 
 /*
  * rpa_profile_enable -- tracing switch (process-wide, default off).  While
- * on, every kernel launch of rpa_forward is bracketed by two CUDA events on
- * the launching stream.  Returns the previous setting.
+ * on, every kernel launch of rpa_forward and rpa_forward_host is bracketed
+ * by two CUDA events on the launching stream (rpa_forward_device and
+ * rpa_decode_noalloc are not traced).  The records accumulate until
+ * rpa_profile_read collects them, so a long traced run should read them
+ * from time to time.  Returns the previous setting.
  */
 RPA_API int32_t rpa_profile_enable(int32_t on);
 
