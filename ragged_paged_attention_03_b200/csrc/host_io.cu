@@ -252,6 +252,10 @@ extern "C" RPA_API int rpa_forward_host(const void *q, const void *k_new, const 
     rc = grow(io, io.io, st.total);
     if (rc) return rc;
     unsigned char *b = io.io.ptr;
+    std::vector<HostPlan> plans(ng);
+    std::vector<int64_t> plan_off(ng + 1, 0), part_off(ng + 1, 0);
+    std::vector<int32_t> cu_g(num_seqs + 1);
+    std::vector<char> has_prefill(ng, 0);
 
     // One group has nothing to overlap: everything runs on the caller's
     // stream, in order, without the event hops between streams.  Otherwise
@@ -293,34 +297,36 @@ extern "C" RPA_API int rpa_forward_host(const void *q, const void *k_new, const 
     if (e == cudaSuccess) e = copy_in(0);
 
     // ---- plan every group (rpa_forward's planner on the group's lengths,
-    // token rows and page-table rows counted from the group start)
-    std::vector<HostPlan> plans(ng);
-    std::vector<int64_t> plan_off(ng + 1, 0), part_off(ng + 1, 0);
-    std::vector<int32_t> cu_g(num_seqs + 1);
-    std::vector<char> has_prefill(ng, 0);
-    for (int g = 0; g < ng; ++g) {
-      const int32_t s0 = bounds[g], ns = bounds[g + 1] - bounds[g];
-      const int32_t t0 = cu_q_lens[s0];
-      for (int32_t s = 0; s <= ns; ++s) {
-        cu_g[s] = cu_q_lens[s0 + s] - t0;
-        if (s > 0 && cu_g[s] - cu_g[s - 1] > 1) has_prefill[g] = 1;
+    // token rows and page-table rows counted from the group start).  Copies
+    // are queued already: a failed host allocation from here on still ends
+    // with the streams joined below.
+    try {
+      for (int g = 0; g < ng; ++g) {
+        const int32_t s0 = bounds[g], ns = bounds[g + 1] - bounds[g];
+        const int32_t t0 = cu_q_lens[s0];
+        for (int32_t s = 0; s <= ns; ++s) {
+          cu_g[s] = cu_q_lens[s0 + s] - t0;
+          if (s > 0 && cu_g[s] - cu_g[s - 1] > 1) has_prefill[g] = 1;
+        }
+        int32_t dist_g[3];
+        const int32_t *dist_p = nullptr;
+        if (distribution) {
+          for (int i = 0; i < 2; ++i) dist_g[i] = std::min(std::max(distribution[i], s0), s0 + ns) - s0;
+          dist_g[2] = ns;
+          dist_p = dist_g;
+        }
+        rpa_dims dg = *dims;
+        dg.total_q_tokens = cu_g[ns];
+        build_plan(cu_g.data(), kv_lens + s0, ns, dist_p, &dg, plans[g]);
+        plan_off[g + 1] = plan_off[g] + ((plans[g].layout.total_words + 63) & ~(int64_t)63);   // 256-byte steps
+        // groups may run concurrently: each has its own partials
+        part_off[g + 1] = part_off[g] + ((plan_partial_floats(plans[g], dg) + 63) & ~(int64_t)63);
       }
-      int32_t dist_g[3];
-      const int32_t *dist_p = nullptr;
-      if (distribution) {
-        for (int i = 0; i < 2; ++i) dist_g[i] = std::min(std::max(distribution[i], s0), s0 + ns) - s0;
-        dist_g[2] = ns;
-        dist_p = dist_g;
-      }
-      rpa_dims dg = *dims;
-      dg.total_q_tokens = cu_g[ns];
-      build_plan(cu_g.data(), kv_lens + s0, ns, dist_p, &dg, plans[g]);
-      plan_off[g + 1] = plan_off[g] + ((plans[g].layout.total_words + 63) & ~(int64_t)63);   // 256-byte steps
-      // groups may run concurrently: each has its own partials
-      part_off[g + 1] = part_off[g] + ((plan_partial_floats(plans[g], dg) + 63) & ~(int64_t)63);
+    } catch (const std::bad_alloc &) {
+      rc = RPA_ERR_OOM;
     }
     const int64_t plan_words = plan_off[ng];
-    if (e == cudaSuccess) rc = grow(io, io.plan, plan_words * 4 + part_off[ng] * 4);
+    if (e == cudaSuccess && rc == RPA_OK) rc = grow(io, io.plan, plan_words * 4 + part_off[ng] * 4);
     PinnedPlan &pin = io.pin[io.next_pin];
     io.next_pin ^= 1;
     if (e == cudaSuccess && rc == RPA_OK) rc = grow_pinned(pin, plan_words);
