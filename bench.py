@@ -6,7 +6,9 @@ update, the decode / prefill kernels, the split-KV combine -- every part of
 the method.  The headline line is the 128-sequence decode batch shaped like a
 Llama-3-8B attention layer (metric: decode HBM GB/s); the prefill (causal and
 not), mixed-batch and head_dim-256 long-context workloads are measured in the
-same run and reported under "also".
+same run.  Each workload prints one short JSON line of its own (value,
+dominant-kernel roofline fraction, end-to-end and CUDA-graph numbers) as it
+finishes; the headline line comes last.
 
 Timing: W untimed warm-up steps, then K steps timed on the device with CUDA
 events on the launching stream, a 256 MiB write between steps to flush the
@@ -17,6 +19,11 @@ once, the page-table entries read once; FLOPs count visible (q, k) pairs only.
 
 ``--impl reference`` times the fp64 CPU oracle instead, on a bounded sample
 of the same workload (the only other place this script runs the oracle).
+
+``--ablate-write`` measures the cost of the fused cache update: every listed
+workload's kernels are timed with this library and, in a child process, with
+a timing-only build whose cache stores are compiled out
+(RPA_ABLATE_CACHE_WRITE); one line per workload gives both kernel times.
 """
 from __future__ import annotations
 
@@ -347,11 +354,13 @@ def roofline(name, work, kern, pk, steps):
         achieved = work["prefill_flops"] / avg_s / 1e12
         r = {"bound": "tensor", "achieved": achieved, "peak": pk["tc"], "unit": "TFLOP/s",
              "peak_source": f"{pk['source']} bf16 dense (burst)"}
+        b = work["bytes"] - work["decode_kernel_bytes"]
     else:
         b = work["decode_kernel_bytes"] if top == "decode" else work["bytes"]
         achieved = b / avg_s / 1e9
         r = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
              "peak_source": f"{pk['source']} HBM copy"}
+    r["alg_bytes"] = b
     r["frac"] = r["achieved"] / r["peak"]
     r["kernel"] = top
     r["kernel_ms"] = total_ms / steps
@@ -409,6 +418,72 @@ def cpu_baseline(name, prob_dev, budget_s):
                       f"{work['flops'] / 1e9:.1f} GFLOP), one fp64 oracle pass, {dt:.1f} s"}
 
 
+# ------------------------------------------------------------ output lines
+def _r(x, digits=4):
+    """x rounded to `digits` significant digits (floats only)."""
+    if isinstance(x, float):
+        return float(f"{x:.{digits}g}") if math.isfinite(x) else x
+    if isinstance(x, dict):
+        return {k: _r(v, digits) for k, v in x.items()}
+    if isinstance(x, list):
+        return [_r(v, digits) for v in x]
+    return x
+
+
+def workload_line(line: dict) -> dict:
+    """The short per-workload line: value, the dominant kernel against its
+    roofline, and the end-to-end and graph-replay values in the same unit."""
+    rf = line["roofline"]
+    short = {"workload": line["workload"], "metric": line["metric"], "value": line["value"],
+             "unit": line["unit"], "ms_per_step": line["ms_per_step"],
+             "roofline": {"kernel": rf["kernel"], "frac": rf["frac"], "achieved": rf["achieved"],
+                          "peak": rf["peak"], "unit": rf["unit"], "kernel_ms": rf["kernel_ms"],
+                          "traffic": rf["traffic"], "alg_bytes": rf.get("alg_bytes")},
+             "e2e": line["e2e"]["value"], "graph": line["device_planned_graph"]["value"]}
+    return _r(short)
+
+
+# --------------------------------------------------- cache-write ablation
+def kernel_times(spec, steps, warmup, dev):
+    """Per kernel class (launches, ms per step) of one workload, kernels run
+    serially (a mixed batch's concurrent schedule would overlap the events)."""
+    from ragged_paged_attention_03_b200 import binding as rb
+    name, _, opt = spec.partition(":")
+    prob = device_problem(name, False if opt == "noncausal" else None, dev)
+    stream = torch.cuda.Stream(dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    old = rb.rpa_set_option(rb.RPA_OPT_CONCURRENT_MIXED, -1)
+    try:
+        ms, kern = time_steps(prob, steps, warmup, flush, stream, profile=True)
+    finally:
+        rb.rpa_set_option(rb.RPA_OPT_CONCURRENT_MIXED, old)
+    return {k: (v[0] / steps, v[1] / steps) for k, v in kern.items() if v[0] > 0}, ms
+
+
+def ablate_write(args, dev):
+    """The fused cache update's cost: each workload's kernel times with the
+    library as built and with the timing-only build whose cache stores are
+    compiled out, run in a child process that loads that build."""
+    from ragged_paged_attention_03_b200 import build
+    build.build()
+    build.build(ablate_write=True)
+    for spec in [w for w in args.workloads.split(",") if w]:
+        with_w, step_w = kernel_times(spec, args.steps, args.warmup, dev)
+        env = dict(os.environ, RPA_ABLATE_CACHE_WRITE="1")
+        r = subprocess.run([sys.executable, os.path.abspath(__file__), "--ablate-child", "--workloads", spec,
+                            "--steps", str(args.steps), "--warmup", str(args.warmup)],
+                           env=env, capture_output=True, text=True, check=True)
+        child = json.loads(r.stdout.strip().splitlines()[-1])
+        without, step_wo = child["kern"], child["ms_per_step"]
+        line = {"ablation": "fused cache write", "workload": spec,
+                "kernel_ms_with_write": {k: v[1] for k, v in with_w.items()},
+                "kernel_ms_without_write": {k: v[1] for k, v in without.items()},
+                "step_ms_with_write": step_w, "step_ms_without_write": step_wo,
+                "write_cost_frac": {k: (with_w[k][1] - without[k][1]) / with_w[k][1]
+                                    for k in with_w if k in without and with_w[k][1] > 0}}
+        print(json.dumps(_r(line)), flush=True)
+
+
 # ----------------------------------------------------------------- main
 def dist_setup(args, backend="nccl"):
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -447,7 +522,22 @@ def main():
     ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
                     help="replicas: every GPU runs the whole batch (weak scaling); heads: every GPU "
                          "runs its Hkv/N KV heads of the same batch (strong scaling; no collective)")
+    ap.add_argument("--ablate-write", action="store_true",
+                    help="time each workload's kernels with and without the fused cache stores "
+                         "(a separate timing-only build; off by default)")
+    ap.add_argument("--ablate-child", action="store_true", help=argparse.SUPPRESS)
     args = ap.parse_args()
+    if args.ablate_write or args.ablate_child:
+        dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+        torch.cuda.set_device(dev)
+        if args.ablate_child:
+            if os.environ.get("RPA_ABLATE_CACHE_WRITE") != "1":
+                raise SystemExit("--ablate-child runs only under RPA_ABLATE_CACHE_WRITE=1")
+            kern, ms = kernel_times(args.workloads.split(",")[0], args.steps, args.warmup, dev)
+            print(json.dumps({"kern": kern, "ms_per_step": ms}), flush=True)
+        elif int(os.environ.get("RANK", "0")) == 0:
+            ablate_write(args, dev)
+        return
     world, rank, local = dist_setup(args)
     n = world
     wl = [w for w in args.workloads.split(",") if w]
@@ -548,6 +638,8 @@ def main():
                                          "host_us_per_host_planned_call": h_host_us}}
         if rank == 0 and i == 0 and world == 1:
             cpu_base = cpu_baseline(name, prob, args.cpu_budget)
+        if rank == 0:
+            print(json.dumps(workload_line(line)), flush=True)
         results.append(line)
         del prob
         torch.cuda.empty_cache()
@@ -563,9 +655,9 @@ def main():
                           (f"KV-head shards x{n}" if args.shard == "heads" else f"replicas x{n}")},
                "roofline": head["roofline"], "e2e": head["e2e"],
                "gpu_launches": head["gpu_launches"], "clocks": clk,
-               "device_planned_graph": head["device_planned_graph"],
-               "cpu_baseline": cpu_base, "also": results[1:]}
-        print(json.dumps(out), flush=True)
+               "cpu_baseline": cpu_base,
+               "workloads": [r["workload"] for r in results]}
+        print(json.dumps(_r(out, 6)), flush=True)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()

@@ -265,10 +265,18 @@ RPA_API int rpa_profile_read(double *ms, int64_t *launches);
  * num_kv_heads * G * (head_dim + 1) floats per split item within ~15.6 MiB).
  * No cudaMalloc, cudaFree, cudaMallocHost or other allocating routine is
  * called.  The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  All calls share the one array and it keeps the
- * last call's contents: calls that can overlap on the GPU race on it, so the
- * caller must order them (for example, one stream per device).
+ * (cudaGetSymbolAddress) and creates one event, with that device current;
+ * make that first call before any stream capture.  All calls share the one
+ * array and it keeps the last call's contents: calls that can overlap on the
+ * GPU race on it, so the caller must order them (for example, one stream per
+ * device).
+ *
+ * The plan is staged in static host arrays and copied with cudaMemcpyAsync;
+ * an event recorded after those copies is waited for by the next call before
+ * it rewrites the arrays, so a call may block until the previous call's plan
+ * copy has run on its stream.  A call on a stream that is being captured
+ * into a CUDA graph returns RPA_ERR_INVALID_ARG before any device work (its
+ * plan would be read from arrays that later calls rewrite).
  */
 RPA_API int rpa_decode_noalloc(const void *q, const void *k_new,
                                const void *v_new, void *k_cache,

@@ -17,7 +17,11 @@ import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "librpa_b200.so")
+# RPA_ABLATE_CACHE_WRITE=1 selects the timing-only build without the fused
+# cache stores (bench.py --ablate-write runs it in a child process); its
+# caches are not updated, so nothing else may use it.
+LIB_PATH = os.path.join(_HERE, "librpa_b200_nowrite.so" if os.environ.get("RPA_ABLATE_CACHE_WRITE") == "1"
+                        else "librpa_b200.so")
 
 RPA_F32, RPA_BF16 = 0, 1
 RPA_OK = 0

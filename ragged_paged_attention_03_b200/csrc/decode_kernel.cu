@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(128) decode_kernel(const __grid_constant__ CUt
           kval = *reinterpret_cast<const uint4 *>(kn + src);
           vval = *reinterpret_cast<const uint4 *>(vn + src);
           const int pg = my_pages[c / P - first_page];
-          if (pg >= 0) {
+          if (kCacheWrite && pg >= 0) {
             const size_t dst = (((size_t)pg * P + c % P) * pb.hkv + hk) * D + ch * 8;
             *reinterpret_cast<uint4 *>(kc + dst) = kval;
             *reinterpret_cast<uint4 *>(vc + dst) = vval;

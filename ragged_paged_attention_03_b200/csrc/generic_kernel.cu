@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(128) generic_kernel(Problem pb, const GenericS
   const int32_t *pt_row = pb.page_table + (size_t)gs.seq * pb.max_pages;
 
   // fused cache update of this token's K/V for KV head hk
-  if (h % G == 0) {
+  if (kCacheWrite && h % G == 0) {
     const int pos = c + i;
     const int page = pt_row[pos / pb.p];
     if (page >= 0 && page < pb.num_pages) {

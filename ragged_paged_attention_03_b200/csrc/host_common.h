@@ -4,6 +4,7 @@
 #pragma once
 #include <stdint.h>
 
+#include "plan.h"
 #include "rpa.h"
 
 namespace rpa {
@@ -21,6 +22,17 @@ int64_t decode_pack_blocks();    // longest packed decode sequence, 0 = never
 int64_t prefill_loaders();       // RPA_OPT_PREFILL_LOADERS as set (0, 1, 2)
 bool concurrent_mixed();         // RPA_OPT_CONCURRENT_MIXED >= 0
 int64_t prefill_sms();           // RPA_OPT_PREFILL_SMS (<= 0: one CTA per SM)
+
+// Decode work items of one sequence with kv_len tokens (one new token at
+// global row `token`): near-equal chunks of at most `chunk` 16-token blocks,
+// decode_items_of(kv_len, chunk) of them.  fill_decode_items writes them to
+// items[0 .. count): the last one owns the new token; when there is more than
+// one, they take partial slots first_partial .. + count - 1 and *combine (if
+// not NULL) receives the combine row that merges them.  Both host planners
+// (rpa_forward's and the allocation-free decode entry point's) call these.
+int32_t decode_items_of(int32_t kv_len, int64_t chunk);
+int32_t fill_decode_items(int32_t seq, int32_t token, int32_t kv_len, int64_t chunk, int32_t first_partial,
+                          DecodeItem *items, CombineItem *combine);
 
 // Packed decode CTAs a batch must fill before packing is used (two per SM
 // of a 148-SM B200): a packed launch follows the main decode launch, so a

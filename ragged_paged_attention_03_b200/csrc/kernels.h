@@ -7,6 +7,18 @@
 
 namespace rpa {
 
+// The fused cache update is on in every product build.  A timing-only build
+// of the library (compiled with RPA_ABLATE_CACHE_WRITE, into a separate file
+// that nothing but the benchmark's --ablate-write leg loads) drops the stores
+// of the new K/V rows, so that their cost inside the attention kernels can be
+// measured; its caches are left unwritten and its results are not the
+// method's.
+#ifdef RPA_ABLATE_CACHE_WRITE
+constexpr bool kCacheWrite = false;
+#else
+constexpr bool kCacheWrite = true;
+#endif
+
 // Device pointers and geometry shared by every kernel of one call.
 struct Problem {
   const void *q;

@@ -36,7 +36,9 @@ namespace {
 // items][partial outputs, fp32][partial lse, fp32].
 constexpr int64_t kScratchBytes = 16ll << 20;
 constexpr int64_t kMaxItems = 8192;      // decode work items
-constexpr int64_t kMaxCombine = 8192;    // sequences needing the combine
+// sequences needing the combine: each has at least two work items, so the
+// item limit keeps them within half of it
+constexpr int64_t kMaxCombine = kMaxItems / 2;
 constexpr int64_t kItemsOff = 256;
 constexpr int64_t kCombineOff = kItemsOff + kMaxItems * (int64_t)sizeof(DecodeItem);
 constexpr int64_t kPartialOff = kCombineOff + kMaxCombine * (int64_t)sizeof(CombineItem);
@@ -47,10 +49,14 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 std::mutex g_mu;
 void *g_scratch_ptr[kMaxDevices] = {};
+// Recorded after each call's plan copies; the next call waits for it before
+// it refills the host staging below.  Created once per device at set-up.
+cudaEvent_t g_staged[kMaxDevices] = {};
+bool g_staged_pending[kMaxDevices] = {};
 
-// Host staging for the plan.  Copies from pageable memory return only after
-// the source has been consumed, so the buffers can be refilled by the next
-// call as soon as cudaMemcpyAsync has returned.
+// Host staging for the plan (pageable, static).  The copies from it are
+// asynchronous; the event above keeps a later call from rewriting it before
+// the copy engine or driver has read it, whenever the driver reads it.
 DecodeItem g_items[kMaxItems];
 CombineItem g_combine[kMaxCombine];
 
@@ -92,8 +98,7 @@ extern "C" RPA_API int rpa_decode_noalloc(const void *q, const void *k_new, cons
   const int64_t chunk = decode_chunk_blocks();
   int64_t n_items = 0, n_partials = 0, n_combine = 0;
   for (int32_t s = 0; s < num_seqs; ++s) {
-    const int64_t nblk = (kv_lens[s] + 15) / 16;
-    const int64_t nsplit = (nblk + chunk - 1) / chunk;
+    const int64_t nsplit = decode_items_of(kv_lens[s], chunk);
     n_items += nsplit;
     if (nsplit > 1) {
       n_partials += nsplit;
@@ -103,45 +108,45 @@ extern "C" RPA_API int rpa_decode_noalloc(const void *q, const void *k_new, cons
   if (n_items > kMaxItems || n_combine > kMaxCombine || n_partials * per_partial > kPartialFloats)
     return RPA_ERR_SCRATCH_LIMIT;
 
+  // The plan goes up from host arrays that the next call rewrites, and the
+  // kernels are sized for this batch: a call recorded into a CUDA graph
+  // would replay whatever plan the arrays hold then.  Refuse capture.
+  cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &capture) != cudaSuccess || capture != cudaStreamCaptureStatusNone)
+    return RPA_ERR_INVALID_ARG;
+
   std::lock_guard<std::mutex> lock(g_mu);
-  // ---- one-time set-up per device: the device address of the array
+  // ---- one-time set-up per device: the device address of the array and
+  // the staging event
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RPA_ERR_CUDA;
   if (g_scratch_ptr[dev] == nullptr) {
     void *ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
       return RPA_ERR_CUDA;
+    if (g_staged[dev] == nullptr &&
+        cudaEventCreateWithFlags(&g_staged[dev], cudaEventDisableTiming) != cudaSuccess)
+      return RPA_ERR_CUDA;
     g_scratch_ptr[dev] = ptr;
   }
   unsigned char *scratch = static_cast<unsigned char *>(g_scratch_ptr[dev]);
+  // the previous call's copies must have read the staging before it changes
+  // (the arrays are shared by every device: wait for each one's last copy)
+  for (int d = 0; d < kMaxDevices; ++d) {
+    if (!g_staged_pending[d]) continue;
+    if (cudaEventSynchronize(g_staged[d]) != cudaSuccess) return RPA_ERR_CUDA;
+    g_staged_pending[d] = false;
+  }
 
-  // ---- plan: near-equal chunks of at most `chunk` 16-token blocks per sequence
+  // ---- plan: near-equal chunks of at most `chunk` 16-token blocks per
+  // sequence, exactly as rpa_forward's planner cuts them
   int32_t ni = 0, nc = 0, np = 0;
   for (int32_t s = 0; s < num_seqs; ++s) {
-    const int32_t kvl = kv_lens[s];
-    const int32_t nblk = (kvl + 15) / 16;
-    const int32_t nsplit = (int32_t)((nblk + chunk - 1) / chunk);
-    const int32_t per = (nblk + nsplit - 1) / nsplit;
-    const int32_t first = np;
-    int32_t made = 0;
-    for (int32_t b = 0; b < nblk; b += per) {
-      DecodeItem &it = g_items[ni++];
-      memset(&it, 0, sizeof it);
-      it.seq = s;
-      it.token = s;
-      it.kv_len = kvl;
-      it.blk_begin = b;
-      it.blk_end = b + per < nblk ? b + per : nblk;
-      it.owns_new = it.blk_end == nblk ? 1 : 0;
-      it.partial = nsplit > 1 ? np++ : -1;
-      ++made;
-    }
+    const int32_t made = fill_decode_items(s, s, kv_lens[s], chunk, np, g_items + ni, g_combine + nc);
+    ni += made;
     if (made > 1) {
-      CombineItem &c = g_combine[nc++];
-      memset(&c, 0, sizeof c);
-      c.token = s;
-      c.first_partial = first;
-      c.nsplit = made;
+      np += made;
+      ++nc;
     }
   }
 
@@ -164,6 +169,8 @@ extern "C" RPA_API int rpa_decode_noalloc(const void *q, const void *k_new, cons
   if (nc > 0 && cudaMemcpyAsync(d_combine, g_combine, (size_t)nc * sizeof(CombineItem),
                                 cudaMemcpyHostToDevice, stream) != cudaSuccess)
     return RPA_ERR_CUDA;
+  if (cudaEventRecord(g_staged[dev], stream) != cudaSuccess) return RPA_ERR_CUDA;
+  g_staged_pending[dev] = true;
 
   Problem pb{};
   pb.q = q;

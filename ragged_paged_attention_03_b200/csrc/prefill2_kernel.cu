@@ -555,6 +555,7 @@ __device__ __forceinline__ void cache_update(const Problem pb, const PrefillTile
                                              int n) {
   using S = P2Shape<D>;
   constexpr int BM = S::BM, BN = S::BN;
+  if (!kCacheWrite) return;
   const int G = pb.hq / pb.hkv;
   const int chunks = D / 8;
   const __nv_bfloat16 *kn = reinterpret_cast<const __nv_bfloat16 *>(pb.k_new);

@@ -350,7 +350,7 @@ __global__ void __launch_bounds__(192, 1)
       // kBatch chunks per thread in flight: the loads (sources and page-table
       // entries) of a batch are issued before its stores
       constexpr int kBatch = 8;
-      const int total = (rb - ra) * chunks;
+      const int total = kCacheWrite ? (rb - ra) * chunks : 0;
       for (int base = tid; base < total; base += 128 * kBatch) {
         uint4 kq[kBatch], vq[kBatch];
         int pgq[kBatch];

@@ -65,6 +65,36 @@ bool concurrent_mixed() { return g_opt_concurrent_mixed.load() >= 0; }
 
 int64_t prefill_sms() { return g_opt_prefill_sms.load(); }
 
+int32_t decode_items_of(int32_t kv_len, int64_t chunk) {
+  const int64_t nblk = ((int64_t)kv_len + kDecodeBlock - 1) / kDecodeBlock;
+  return (int32_t)((nblk + chunk - 1) / chunk);
+}
+
+int32_t fill_decode_items(int32_t seq, int32_t token, int32_t kv_len, int64_t chunk, int32_t first_partial,
+                          DecodeItem *items, CombineItem *combine) {
+  const int32_t nblk = (kv_len + kDecodeBlock - 1) / kDecodeBlock;
+  const int32_t nsplit = decode_items_of(kv_len, chunk);
+  const int32_t per = (nblk + nsplit - 1) / nsplit;   // ceil(nblk / per) == nsplit
+  for (int32_t k = 0; k < nsplit; ++k) {
+    DecodeItem &it = items[k];
+    memset(&it, 0, sizeof it);
+    it.seq = seq;
+    it.token = token;
+    it.kv_len = kv_len;
+    it.blk_begin = k * per;
+    it.blk_end = std::min(nblk, it.blk_begin + per);
+    it.owns_new = it.blk_end == nblk ? 1 : 0;
+    it.partial = nsplit > 1 ? first_partial + k : -1;
+  }
+  if (nsplit > 1 && combine != nullptr) {
+    memset(combine, 0, sizeof *combine);
+    combine->token = token;
+    combine->first_partial = first_partial;
+    combine->nsplit = nsplit;
+  }
+  return nsplit;
+}
+
 int validate_dims(const rpa_dims *d) {
   if (d == nullptr) return RPA_ERR_INVALID_ARG;
   if (d->num_q_heads <= 0 || d->num_kv_heads <= 0 || d->num_pages <= 0 ||
@@ -165,28 +195,14 @@ void build_plan(const int32_t *cu, const int32_t *kv, int32_t n, const int32_t *
           hp.decode_max_splits = std::max(hp.decode_max_splits, 1);
           break;
         }
-        const int32_t nsplit = (int32_t)((nblk + chunk - 1) / chunk);
-        const int32_t per = (nblk + nsplit - 1) / nsplit;
+        const int32_t nsplit = decode_items_of(kvl, chunk);
         hp.decode_max_splits = std::max(hp.decode_max_splits, nsplit);
-        const int32_t first_partial = hp.n_partials;
-        int32_t made = 0;
-        for (int32_t b = 0; b < nblk; b += per) {
-          DecodeItem it{};
-          it.seq = s;
-          it.token = cu[s];
-          it.kv_len = kvl;
-          it.blk_begin = b;
-          it.blk_end = std::min(nblk, b + per);
-          it.owns_new = it.blk_end == nblk ? 1 : 0;
-          it.partial = nsplit > 1 ? hp.n_partials++ : -1;
-          hp.decode.push_back(it);
-          ++made;
-        }
-        if (made > 1) {
-          CombineItem c{};
-          c.token = cu[s];
-          c.first_partial = first_partial;
-          c.nsplit = made;
+        const size_t at = hp.decode.size();
+        hp.decode.resize(at + (size_t)nsplit);
+        CombineItem c{};
+        fill_decode_items(s, cu[s], kvl, chunk, hp.n_partials, hp.decode.data() + at, &c);
+        if (nsplit > 1) {
+          hp.n_partials += nsplit;
           hp.combine.push_back(c);
         }
         break;

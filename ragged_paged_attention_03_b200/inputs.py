@@ -147,29 +147,56 @@ def make_workload(name: str, device="cpu", causal: Optional[bool] = None, poison
                   head_shard: Optional[Tuple[int, int]] = None) -> Problem:
     """One of the named workloads (see the module docstring).  ``max_seqs``
     keeps only the first sequences (smaller cases for profiler captures).
-    ``head_shard = (rank, n)``: rank's share of a KV-head split over n GPUs:
-    the same sequences and lengths, Hkv / n KV heads with their Hq / n query
-    heads (heads never interact, so the shards need no exchange); values are
-    drawn with a rank-specific seed."""
+    ``head_shard = (rank, n)``: rank's share of a KV-head split of the same
+    batch over n GPUs (``head_slice`` of the whole draw): Hkv / n KV heads with
+    their Hq / n query heads, every sequence, length and page (heads never
+    interact, so the shards need no exchange)."""
     dtype, hq, hkv, d, p, causal_default, vscale, seed, pool = WORKLOADS[name]
     if head_shard is not None:
         rank, n = head_shard
         if n < 1 or hkv % n != 0 or not 0 <= rank < n:
             raise ValueError(f"{name}: {hkv} KV heads do not split over {n} GPUs")
-        hq, hkv = hq // n, hkv // n
     gen = torch.Generator().manual_seed(seed)
     q_lens, kv_lens = _lengths(name, gen)
     if max_seqs is not None:
         q_lens, kv_lens = q_lens[:max_seqs], kv_lens[:max_seqs]
     if logical is None:
         logical = name == "tiny_mixed_f32"
-    if head_shard is not None and head_shard[0] > 0:
-        seed = seed + 7919 * head_shard[0]   # the lengths above are shared; pages and values per shard
-        gen.manual_seed(seed)
-    return make_problem(q_lens, kv_lens, num_q_heads=hq, num_kv_heads=hkv, head_dim=d,
+    prob = make_problem(q_lens, kv_lens, num_q_heads=hq, num_kv_heads=hkv, head_dim=d,
                         page_size=p, dtype=dtype, causal=causal_default if causal is None else causal,
                         seed=seed, pool=pool, value_scale=vscale, device=device, poison=poison,
                         logical=logical, name=name, gen=gen)
+    if head_shard is None or head_shard[1] == 1:
+        return prob
+    shard = head_slice(prob, *head_shard)
+    del prob
+    return shard
+
+
+def head_slice(prob: Problem, rank: int, n: int) -> Problem:
+    """KV heads [rank * Hkv / n, (rank + 1) * Hkv / n) of a problem, with
+    their query heads (query head h reads KV head h // G, so they are the
+    matching contiguous range): q, k_new, v_new and both caches sliced along
+    the head axis into contiguous copies; lengths, pages, page table, scale
+    and mask unchanged."""
+    hkv, hq = prob.num_kv_heads, prob.num_q_heads
+    if n < 1 or hkv % n != 0 or not 0 <= rank < n:
+        raise ValueError(f"{hkv} KV heads do not split {n} ways")
+    kv0, kv1 = rank * hkv // n, (rank + 1) * hkv // n
+    g = hq // hkv
+    q0, q1 = kv0 * g, kv1 * g
+
+    def cut(t, a, b, axis):
+        return t.narrow(axis, a, b - a).contiguous()
+
+    d = dict(prob.__dict__)
+    d.update(num_q_heads=q1 - q0, num_kv_heads=kv1 - kv0,
+             q=cut(prob.q, q0, q1, 1), k_new=cut(prob.k_new, kv0, kv1, 1), v_new=cut(prob.v_new, kv0, kv1, 1),
+             k_cache=cut(prob.k_cache, kv0, kv1, 2), v_cache=cut(prob.v_cache, kv0, kv1, 2),
+             ctx_k=None if prob.ctx_k is None else [cut(t, kv0, kv1, 1) for t in prob.ctx_k],
+             ctx_v=None if prob.ctx_v is None else [cut(t, kv0, kv1, 1) for t in prob.ctx_v],
+             meta={**prob.meta, "head_shard": (rank, n)})
+    return Problem(**d)
 
 
 def make_problem(q_lens: Sequence[int], kv_lens: Sequence[int], *, num_q_heads: int,

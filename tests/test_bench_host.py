@@ -110,17 +110,23 @@ def test_roofline_uses_the_dominant_kernel():
 
 
 def test_head_shards_split_heads_not_sequences():
-    """--shard heads: each rank gets the same sequences with Hkv / n KV heads
-    and their query heads; n must divide Hkv."""
+    """--shard heads: each rank gets the same sequences, lengths and pages
+    with Hkv / n KV heads and their query heads, sliced from the one batch
+    (concatenated along the head axis, the shards give back the whole draw);
+    n must divide Hkv."""
     full = I.make_workload("tiny_mixed_f32", device="cpu")
     shards = [I.make_workload("mixed_96d_4c", device="cpu", poison=False, head_shard=(r, 4), max_seqs=6)
               for r in range(4)]
     ref = I.make_workload("mixed_96d_4c", device="cpu", poison=False, max_seqs=6)
     for sh in shards:
         assert list(sh.q_lens) == list(ref.q_lens) and list(sh.kv_lens) == list(ref.kv_lens)
+        assert torch.equal(sh.page_table, ref.page_table)
         assert sh.q.shape == (ref.q.shape[0], ref.q.shape[1] // 4, ref.q.shape[2])
         assert sh.k_cache.shape[2] == ref.k_cache.shape[2] // 4
-    assert not torch.equal(shards[0].q, shards[1].q)          # rank-specific values
+        assert sh.q.is_contiguous() and sh.k_cache.is_contiguous()
+    for name, axis in (("q", 1), ("k_new", 1), ("v_new", 1), ("k_cache", 2), ("v_cache", 2)):
+        whole = torch.cat([getattr(sh, name) for sh in shards], dim=axis)
+        assert torch.equal(whole.view(torch.int16), getattr(ref, name).view(torch.int16)), name
     with pytest.raises(ValueError):
         I.make_workload("tiny_mixed_f32", device="cpu", head_shard=(0, 2))   # 1 KV head
     assert full.q.shape[1] == 4
