@@ -522,6 +522,9 @@ def main():
     ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
                     help="replicas: every GPU runs the whole batch (weak scaling); heads: every GPU "
                          "runs its Hkv/N KV heads of the same batch (strong scaling; no collective)")
+    ap.add_argument("--prefill-kernel", type=int, default=None,
+                    help="RPA_OPT_PREFILL_KERNEL for the head_dim 128 prefill (0 or 1: two tiles per CTA, "
+                         "the default; 2: CTA pairs; 3: one tile per CTA)")
     ap.add_argument("--ablate-write", action="store_true",
                     help="time each workload's kernels with and without the fused cache stores "
                          "(a separate timing-only build; off by default)")
@@ -540,6 +543,9 @@ def main():
         return
     world, rank, local = dist_setup(args)
     n = world
+    if args.prefill_kernel is not None:
+        from ragged_paged_attention_03_b200 import binding as rb
+        rb.rpa_set_option(rb.RPA_OPT_PREFILL_KERNEL, args.prefill_kernel)
     wl = [w for w in args.workloads.split(",") if w]
 
     if args.impl == "reference":

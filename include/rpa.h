@@ -209,13 +209,22 @@ enum {
                                       instead of two), 0 = chosen per batch:
                                       2 when the prefill rows' cached context
                                       outnumbers their new tokens (default 0) */
-  RPA_OPT_DECODE_PACK_BLOCKS = 6   /* decode sequences of at most this many
+  RPA_OPT_DECODE_PACK_BLOCKS = 6,  /* decode sequences of at most this many
                                       16-token blocks (and within one work
                                       item) run four per CTA, one per warp,
                                       when they make at least 296 such CTAs
                                       (two per SM); fewer stay in the main
                                       decode launch (default 64; 0 restores
                                       it, < 0: never) */
+  RPA_OPT_PREFILL_KERNEL = 7       /* head_dim 128 prefill kernel: 0 (default)
+                                      or 1 two 128-row tiles per CTA (the
+                                      head_dim 64 kernel); 2 CTA pairs
+                                      sharing M = 256 tcgen05 MMAs, one
+                                      256-row item per pair, three score
+                                      buffers; 3 the same with one 128-row
+                                      tile per CTA.  Results agree within
+                                      rounding; 2 and 3 measured slower and
+                                      are kept for measurement */
 };
 RPA_API int64_t rpa_set_option(int32_t option, int64_t value);
 

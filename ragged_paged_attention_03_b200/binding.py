@@ -34,6 +34,7 @@ RPA_OPT_PREFILL_SMS = 3
 RPA_OPT_CONCURRENT_MIXED = 4
 RPA_OPT_PREFILL_LOADERS = 5
 RPA_OPT_DECODE_PACK_BLOCKS = 6
+RPA_OPT_PREFILL_KERNEL = 7
 
 
 class rpa_dims(ctypes.Structure):

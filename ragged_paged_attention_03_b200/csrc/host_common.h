@@ -4,6 +4,7 @@
 #pragma once
 #include <stdint.h>
 
+#include "kernels.h"
 #include "plan.h"
 #include "rpa.h"
 
@@ -22,6 +23,12 @@ int64_t decode_pack_blocks();    // longest packed decode sequence, 0 = never
 int64_t prefill_loaders();       // RPA_OPT_PREFILL_LOADERS as set (0, 1, 2)
 bool concurrent_mixed();         // RPA_OPT_CONCURRENT_MIXED >= 0
 int64_t prefill_sms();           // RPA_OPT_PREFILL_SMS (<= 0: one CTA per SM)
+int64_t prefill_kernel();        // RPA_OPT_PREFILL_KERNEL as set (0 .. 3)
+
+// The prefill kernel for this head dim (RPA_OPT_PREFILL_KERNEL picks among
+// the head_dim 128 ones): the same launch contract as launch_prefill2.
+cudaError_t launch_prefill_any(const Problem &pb, const PrefillTile *tiles, int n_tiles, int max_ctas, bool split,
+                               cudaStream_t stream);
 
 // Decode work items of one sequence with kv_len tokens (one new token at
 // global row `token`): near-equal chunks of at most `chunk` 16-token blocks,

@@ -66,6 +66,13 @@ cudaError_t launch_prefill(const Problem &pb, const PrefillTile *tiles,
 cudaError_t launch_prefill2(const Problem &pb, const PrefillTile *tiles,
                             int n_tiles, int max_ctas, bool split, cudaStream_t stream);
 
+// head_dim 128 with a double-buffered score tile: persistent; pair: CTA
+// pairs (clusters of two) sharing M = 256 MMAs, one 256-row work item per
+// pair; otherwise one CTA per 128-row half of an item.  At most max_ctas
+// CTAs (<= 0: as many as fit, one per SM).
+cudaError_t launch_prefill3(const Problem &pb, const PrefillTile *tiles,
+                            int n_tiles, int max_ctas, bool pair, cudaStream_t stream);
+
 // Rows of a single prefill tile (query tokens per TMEM accumulator).
 constexpr int kPrefillTileRows = 128;
 

@@ -34,6 +34,7 @@ std::atomic<int64_t> g_opt_prefill_sms{0};
 std::atomic<int64_t> g_opt_concurrent_mixed{0};
 std::atomic<int64_t> g_opt_prefill_loaders{0};
 std::atomic<int64_t> g_opt_decode_pack{0};
+std::atomic<int64_t> g_opt_prefill_kernel{0};
 
 constexpr int kDefaultDecodeChunkBlocks = 192;
 // Decode sequences this short (16-token blocks) run four per CTA, one per
@@ -64,6 +65,16 @@ int64_t prefill_loaders() { return g_opt_prefill_loaders.load(); }
 bool concurrent_mixed() { return g_opt_concurrent_mixed.load() >= 0; }
 
 int64_t prefill_sms() { return g_opt_prefill_sms.load(); }
+
+int64_t prefill_kernel() { return g_opt_prefill_kernel.load(); }
+
+cudaError_t launch_prefill_any(const Problem &pb, const PrefillTile *tiles, int n_tiles, int max_ctas, bool split,
+                               cudaStream_t stream) {
+  if (pb.d == 256) return launch_prefill(pb, tiles, n_tiles, stream);
+  const int64_t k = prefill_kernel();
+  if (pb.d == 128 && (k == 2 || k == 3)) return launch_prefill3(pb, tiles, n_tiles, max_ctas, k == 2, stream);
+  return launch_prefill2(pb, tiles, n_tiles, max_ctas, split, stream);
+}
 
 int32_t decode_items_of(int32_t kv_len, int64_t chunk) {
   const int64_t nblk = ((int64_t)kv_len + kDecodeBlock - 1) / kDecodeBlock;
@@ -457,8 +468,7 @@ cudaError_t launch_kernels(DeviceWs &ws, const HostPlan &hp, const int32_t *dev_
       // per operand; fresh prefill keeps two warps for the cache update
       const int64_t lo = g_opt_prefill_loaders.load();
       const bool split = lo == 2 || (lo != 1 && hp.prefill_ctx_tokens > hp.prefill_new_tokens);
-      return pb.d <= 128 ? launch_prefill2(pb, tiles, (int)L.n_prefill_tiles, prefill_ctas, split, pstream)
-                         : launch_prefill(pb, tiles, (int)L.n_prefill_tiles, pstream);
+      return launch_prefill_any(pb, tiles, (int)L.n_prefill_tiles, prefill_ctas, split, pstream);
     });
   if (mixed && cudaEventRecord(join, pstream) != cudaSuccess) e = cudaErrorUnknown;
   if (L.n_decode_items > 0 && e == cudaSuccess)
@@ -558,6 +568,7 @@ extern "C" RPA_API int64_t rpa_set_option(int32_t option, int64_t value) {
     case RPA_OPT_CONCURRENT_MIXED: return g_opt_concurrent_mixed.exchange(value);
     case RPA_OPT_PREFILL_LOADERS: return g_opt_prefill_loaders.exchange(value);
     case RPA_OPT_DECODE_PACK_BLOCKS: return g_opt_decode_pack.exchange(value);
+    case RPA_OPT_PREFILL_KERNEL: return g_opt_prefill_kernel.exchange(value);
     default: return -1;
   }
 }
