@@ -285,6 +285,9 @@ __device__ __forceinline__ void produce_kv(Bars2 *bars, volatile int *abort_flag
   constexpr int BM = S::BM, BN = S::BN, NSK = S::NSK, NSV = S::NSV;
   const CUtensorMap &tm_q = *tmq, &tm_kc = *tmkc, &tm_vc = *tmvc, &tm_kn = *tmkn, &tm_vn = *tmvn;
   const int lane = threadIdx.x & 31;
+  // Q tiles are read once: first out of L2, ahead of the K/V blocks that
+  // the other query heads of the KV head read again
+  const uint64_t once = ptx::l2_evict_first_policy();
   const int br = pb.p < BN ? pb.p : BN;
   const int nseg = BN / br;
   uint32_t fix_phase = 0;
@@ -305,8 +308,8 @@ __device__ __forceinline__ void produce_kv(Bars2 *bars, volatile int *abort_flag
     for (int t = 0; t < 2; ++t) {
       if (w.rows_t[t] == 0) continue;
       for (int hh = 0; hh < S::kHalves; ++hh)
-        ptx::tma_load_3d_elect(sQ + t * S::kQBytes + hh * BM * 128, &tm_q, &bars->q_full, hh * 64, w.h,
-                               w.tile.q_start + w.r0 + t * BM);
+        ptx::tma_load_3d_hint_elect(sQ + t * S::kQBytes + hh * BM * 128, &tm_q, &bars->q_full, hh * 64, w.h,
+                                    w.tile.q_start + w.r0 + t * BM, once);
     }
     // page of this lane's segment of context block j (-1: no segment);
     // block j+1's entries are read while block j is issued
@@ -441,6 +444,7 @@ __device__ __forceinline__ void produce(Bars2 *bars, volatile int *abort_flag, c
   uint64_t *empty = IS_V ? bars->v_empty : bars->k_empty;
   uint64_t *fixb = &bars->fix[IS_V ? 1 : 0];
   const int lane = threadIdx.x & 31;
+  const uint64_t once = ptx::l2_evict_first_policy();   // for the Q tiles (read once)
   const int br = pb.p < BN ? pb.p : BN;
   const int nseg = BN / br;
   uint32_t fix_phase = 0;
@@ -462,8 +466,8 @@ __device__ __forceinline__ void produce(Bars2 *bars, volatile int *abort_flag, c
       for (int t = 0; t < 2; ++t) {
         if (w.rows_t[t] == 0) continue;
         for (int hh = 0; hh < S::kHalves; ++hh)
-          ptx::tma_load_3d_elect(sQ + t * S::kQBytes + hh * BM * 128, tm_q, &bars->q_full, hh * 64, w.h,
-                                 w.tile.q_start + w.r0 + t * BM);
+          ptx::tma_load_3d_hint_elect(sQ + t * S::kQBytes + hh * BM * 128, tm_q, &bars->q_full, hh * 64, w.h,
+                                      w.tile.q_start + w.r0 + t * BM, once);
       }
     }
     // page of this lane's segment of context block j (-1: no such segment)
@@ -816,13 +820,14 @@ __global__ void __launch_bounds__(384, 1)
       ptx::tc_fence_before();
       ptx::mbar_arrive(&bars->o_free[t]);
       if (store) {
+        const uint64_t once = ptx::l2_evict_first_policy();   // written once: first out of L2
 #pragma unroll
         for (int cc = 0; cc < D / 8; ++cc) {
           uint32_t o2[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             o2[i] = ptx::pack_bf16(__uint_as_float(ov[cc * 8 + 2 * i]) * inv, __uint_as_float(ov[cc * 8 + 2 * i + 1]) * inv);
-          reinterpret_cast<uint4 *>(out)[cc] = make_uint4(o2[0], o2[1], o2[2], o2[3]);
+          ptx::st_global_hint(reinterpret_cast<uint4 *>(out) + cc, make_uint4(o2[0], o2[1], o2[2], o2[3]), once);
         }
       }
       ++ep;

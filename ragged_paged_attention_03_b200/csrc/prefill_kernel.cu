@@ -168,8 +168,11 @@ __global__ void __launch_bounds__(192, 1)
     int gk = 0, gv = 0;                        // blocks whose K (V) copies were queued and published
     bool fix_pending = false;
     ptx::mbar_arrive_expect_tx_elect(&bars->q_full, S::kQBytes);
+    // Q is read once: first out of L2, ahead of the K/V blocks that the
+    // other query heads and later tiles of the sequence read again
+    const uint64_t once = ptx::l2_evict_first_policy();
     for (int hh = 0; hh < S::kHalves; ++hh)
-      ptx::tma_load_3d_elect(sQ + hh * BM * 128, &tm_q, &bars->q_full, hh * 64, h, tile.q_start + r0);
+      ptx::tma_load_3d_hint_elect(sQ + hh * BM * 128, &tm_q, &bars->q_full, hh * 64, h, tile.q_start + r0, once);
     for (int j = 0; j < nb; ++j) {
       const int sk = j % NSK, sv = j % NSV;
       const uint32_t phk = (uint32_t)((j / NSK) & 1), phv = (uint32_t)((j / NSV) & 1);
@@ -487,6 +490,7 @@ __global__ void __launch_bounds__(192, 1)
       ptx::tc_fence_after();
       const float inv = 1.f / l;
       const bool store = row < tile.rows;
+      const uint64_t once = ptx::l2_evict_first_policy();   // written once: first out of L2
       __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(pb.out) +
                            ((size_t)(tile.q_start + rn) * pb.hq + h) * D;
 #pragma unroll
@@ -501,7 +505,8 @@ __global__ void __launch_bounds__(192, 1)
             pk[i] = ptx::pack_bf16(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
           uint4 *dst = reinterpret_cast<uint4 *>(out + cc * 32);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          for (int i = 0; i < 4; ++i)
+            ptx::st_global_hint(dst + i, make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]), once);
         }
       }
       if (store && pb.lse != nullptr) pb.lse[(size_t)(tile.q_start + rn) * pb.hq + h] = (m + log2f(l)) * kLn2;
