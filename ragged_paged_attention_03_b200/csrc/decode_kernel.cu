@@ -29,6 +29,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <math.h>
+#include <string.h>
 
 #include "kernels.h"
 #include "ptx.cuh"
@@ -62,12 +63,14 @@ __device__ __forceinline__ uint32_t tile_off(int r, int ch) {
 // warp) -- short sequences, several per CTA -- and writes its result from
 // registers; otherwise the four warps share one item and merge at the end.
 template <int D, int NG, bool PACK>
-__global__ void __launch_bounds__(128) decode_kernel(const __grid_constant__ CUtensorMap tm_k,
-                                                     const __grid_constant__ CUtensorMap tm_v,
-                                                     const Problem pb, const DecodeItem *__restrict__ items,
-                                                     int n_items, float *__restrict__ part_o,
-                                                     float *__restrict__ part_lse, float scale_log2) {
+__device__ __forceinline__ void decode_body(const CUtensorMap &tm_k, const CUtensorMap &tm_v, const Problem &pb,
+                                            const DecodeItem *__restrict__ items, int n_items,
+                                            float *__restrict__ part_o, float *__restrict__ part_lse,
+                                            float scale_log2) {
   using S = DecodeShape<D>;
+  // a split-KV combine queued behind this grid may be scheduled as soon as
+  // every CTA of it has started; it waits for this grid's results itself
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   constexpr int NST = S::kStages;
   constexpr int KS = D / 16;  // k-steps of QK^T, m-tiles of PV
   extern __shared__ uint8_t smem_raw[];
@@ -427,13 +430,41 @@ __global__ void __launch_bounds__(128) decode_kernel(const __grid_constant__ CUt
   }
 }
 
+template <int D, int NG, bool PACK>
+__global__ void __launch_bounds__(128) decode_kernel(const __grid_constant__ CUtensorMap tm_k,
+                                                     const __grid_constant__ CUtensorMap tm_v,
+                                                     const Problem pb, const DecodeItem *__restrict__ items,
+                                                     int n_items, float *__restrict__ part_o,
+                                                     float *__restrict__ part_lse, float scale_log2) {
+  decode_body<D, NG, PACK>(tm_k, tm_v, pb, items, n_items, part_o, part_lse, scale_log2);
+}
+
+// The work items of a small host-planned decode batch, passed by value in the
+// launch itself, so that no plan copy has to reach the device first.
+constexpr int kInlineItems = 900;    // 28.8 KB of kernel parameters
+struct DecodeInline {
+  DecodeItem items[kInlineItems];
+};
+
+template <int D, int NG>
+__global__ void __launch_bounds__(128) decode_inline_kernel(const __grid_constant__ CUtensorMap tm_k,
+                                                            const __grid_constant__ CUtensorMap tm_v,
+                                                            const Problem pb, const __grid_constant__ DecodeInline plan,
+                                                            int n_items, float *__restrict__ part_o,
+                                                            float *__restrict__ part_lse, float scale_log2) {
+  decode_body<D, NG, false>(tm_k, tm_v, pb, plan.items, n_items, part_o, part_lse, scale_log2);
+}
+
 // One warp per (sequence, query head): merge the normalised partial outputs
 // of the sequence's chunks with weights exp(lse_i - lse), lse = log sum exp.
 template <int D>
-__global__ void __launch_bounds__(128) combine_kernel(const Problem pb, const CombineItem *__restrict__ items,
-                                                      int n_items, const float *__restrict__ part_o,
-                                                      const float *__restrict__ part_lse) {
+__device__ __forceinline__ void combine_body(const Problem &pb, const CombineItem *__restrict__ items,
+                                             int n_items, const float *__restrict__ part_o,
+                                             const float *__restrict__ part_lse) {
   constexpr int E = D / 32;
+  // launched right behind the decode grid (programmatic dependent launch):
+  // its partial results are complete and visible after this wait
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (pb.dev_counts != nullptr) n_items = min(n_items, pb.dev_counts[kCntCombine]);
@@ -472,23 +503,82 @@ __global__ void __launch_bounds__(128) combine_kernel(const Problem pb, const Co
   if (lane == 0 && pb.lse != nullptr) pb.lse[(size_t)ci.token * pb.hq + h] = mstar + logf(wsum);
 }
 
+template <int D>
+__global__ void __launch_bounds__(128) combine_kernel(const Problem pb, const CombineItem *__restrict__ items,
+                                                      int n_items, const float *__restrict__ part_o,
+                                                      const float *__restrict__ part_lse) {
+  combine_body<D>(pb, items, n_items, part_o, part_lse);
+}
+
+constexpr int kInlineRows = 1800;   // 28.8 KB of kernel parameters
+struct CombineInline {
+  CombineItem rows[kInlineRows];
+};
+
+template <int D>
+__global__ void __launch_bounds__(128) combine_inline_kernel(const Problem pb, const __grid_constant__ CombineInline plan,
+                                                             int n_items, const float *__restrict__ part_o,
+                                                             const float *__restrict__ part_lse) {
+  combine_body<D>(pb, plan.rows, n_items, part_o, part_lse);
+}
+
+bool decode_maps(const Problem &pb, int D, CUtensorMap *tk, CUtensorMap *tv) {
+  const uint64_t dims[3] = {(uint64_t)D, (uint64_t)pb.hkv, (uint64_t)pb.num_pages * pb.p};
+  const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)pb.hkv * D * 2};
+  const uint32_t box[3] = {64, 1, (uint32_t)(pb.p < 16 ? pb.p : 16)};
+  return make_tmap_bf16_3d(tk, pb.k_cache, dims, strides, box, true) &&
+         make_tmap_bf16_3d(tv, pb.v_cache, dims, strides, box, true);
+}
+
 template <int D, int NG, bool PACK>
 cudaError_t launch_decode_t(const Problem &pb, const DecodeItem *items, int n_items, float *po, float *pl,
                             cudaStream_t stream) {
   using S = DecodeShape<D>;
   CUtensorMap tk, tv;
-  const uint64_t dims[3] = {(uint64_t)D, (uint64_t)pb.hkv, (uint64_t)pb.num_pages * pb.p};
-  const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)pb.hkv * D * 2};
-  const uint32_t box[3] = {64, 1, (uint32_t)(pb.p < 16 ? pb.p : 16)};
-  if (!make_tmap_bf16_3d(&tk, pb.k_cache, dims, strides, box, true) ||
-      !make_tmap_bf16_3d(&tv, pb.v_cache, dims, strides, box, true))
-    return cudaErrorInvalidValue;
+  if (!decode_maps(pb, D, &tk, &tv)) return cudaErrorInvalidValue;
   auto kern = decode_kernel<D, NG, PACK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)(PACK ? (n_items + kWarps - 1) / kWarps : n_items), (unsigned)pb.hkv);
   kern<<<grid, kWarps * 32, S::kSmem, stream>>>(tk, tv, pb, items, n_items, po, pl, pb.scale * kLog2e);
   return cudaGetLastError();
+}
+
+template <int D, int NG>
+cudaError_t launch_decode_inline_t(const Problem &pb, const DecodeItem *host_items, int n_items, float *po,
+                                   float *pl, cudaStream_t stream) {
+  using S = DecodeShape<D>;
+  CUtensorMap tk, tv;
+  if (!decode_maps(pb, D, &tk, &tv)) return cudaErrorInvalidValue;
+  auto kern = decode_inline_kernel<D, NG>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem);
+  if (e != cudaSuccess) return e;
+  static thread_local DecodeInline plan;   // parameter staging (the launch copies it)
+  memcpy(plan.items, host_items, (size_t)n_items * sizeof(DecodeItem));
+  dim3 grid((unsigned)n_items, (unsigned)pb.hkv);
+  kern<<<grid, kWarps * 32, S::kSmem, stream>>>(tk, tv, pb, plan, n_items, po, pl, pb.scale * kLog2e);
+  return cudaGetLastError();
+}
+
+// The combine queued right behind the decode grid with programmatic
+// dependent launch (when `pdl`): its CTAs may start during the decode tail
+// and wait on the device for the decode results.
+template <typename K, typename... Args>
+cudaError_t launch_combine_grid(K kern, unsigned blocks, bool pdl, cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(blocks, 1, 1);
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  if (pdl) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace
@@ -515,17 +605,52 @@ cudaError_t launch_decode(const Problem &pb, const DecodeItem *items, int n_item
 }
 
 cudaError_t launch_combine(const Problem &pb, const CombineItem *items, int n_items, const float *partial_o,
-                           const float *partial_lse, cudaStream_t stream) {
+                           const float *partial_lse, cudaStream_t stream, bool pdl) {
   if (n_items <= 0) return cudaSuccess;
   const long long warps = (long long)n_items * pb.hq;
   const unsigned blocks = (unsigned)((warps + 3) / 4);
   switch (pb.d) {
-    case 64: combine_kernel<64><<<blocks, 128, 0, stream>>>(pb, items, n_items, partial_o, partial_lse); break;
-    case 128: combine_kernel<128><<<blocks, 128, 0, stream>>>(pb, items, n_items, partial_o, partial_lse); break;
-    case 256: combine_kernel<256><<<blocks, 128, 0, stream>>>(pb, items, n_items, partial_o, partial_lse); break;
+    case 64: return launch_combine_grid(combine_kernel<64>, blocks, pdl, stream, pb, items, n_items, partial_o, partial_lse);
+    case 128: return launch_combine_grid(combine_kernel<128>, blocks, pdl, stream, pb, items, n_items, partial_o, partial_lse);
+    case 256: return launch_combine_grid(combine_kernel<256>, blocks, pdl, stream, pb, items, n_items, partial_o, partial_lse);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
+}
+
+bool decode_plan_fits_inline(int n_items, int n_combine) {
+  return n_items <= kInlineItems && n_combine <= kInlineRows;
+}
+
+cudaError_t launch_decode_inline(const Problem &pb, const DecodeItem *host_items, int n_items, float *partial_o,
+                                 float *partial_lse, cudaStream_t stream) {
+  if (n_items <= 0) return cudaSuccess;
+  if (n_items > kInlineItems) return cudaErrorInvalidValue;
+  const bool two = pb.hq / pb.hkv > 8;
+  switch (pb.d) {
+    case 64: return two ? launch_decode_inline_t<64, 2>(pb, host_items, n_items, partial_o, partial_lse, stream)
+                        : launch_decode_inline_t<64, 1>(pb, host_items, n_items, partial_o, partial_lse, stream);
+    case 128: return two ? launch_decode_inline_t<128, 2>(pb, host_items, n_items, partial_o, partial_lse, stream)
+                         : launch_decode_inline_t<128, 1>(pb, host_items, n_items, partial_o, partial_lse, stream);
+    case 256: return two ? launch_decode_inline_t<256, 2>(pb, host_items, n_items, partial_o, partial_lse, stream)
+                         : launch_decode_inline_t<256, 1>(pb, host_items, n_items, partial_o, partial_lse, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_combine_inline(const Problem &pb, const CombineItem *host_rows, int n_items,
+                                  const float *partial_o, const float *partial_lse, cudaStream_t stream, bool pdl) {
+  if (n_items <= 0) return cudaSuccess;
+  if (n_items > kInlineRows) return cudaErrorInvalidValue;
+  static thread_local CombineInline plan;   // parameter staging (the launch copies it)
+  memcpy(plan.rows, host_rows, (size_t)n_items * sizeof(CombineItem));
+  const long long warps = (long long)n_items * pb.hq;
+  const unsigned blocks = (unsigned)((warps + 3) / 4);
+  switch (pb.d) {
+    case 64: return launch_combine_grid(combine_inline_kernel<64>, blocks, pdl, stream, pb, plan, n_items, partial_o, partial_lse);
+    case 128: return launch_combine_grid(combine_inline_kernel<128>, blocks, pdl, stream, pb, plan, n_items, partial_o, partial_lse);
+    case 256: return launch_combine_grid(combine_inline_kernel<256>, blocks, pdl, stream, pb, plan, n_items, partial_o, partial_lse);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace rpa

@@ -436,7 +436,7 @@ extern "C" RPA_API int rpa_forward_device(const void *q, const void *k_new, cons
     if (e == cudaSuccess && L.cap_packed > 0)
       e = launch_decode(pb, a.packed, (int)L.cap_packed, part_o, part_lse, true, stream);
     if (e == cudaSuccess && L.cap_combine > 0)
-      e = launch_combine(pb, a.combine, (int)L.cap_combine, part_o, part_lse, stream);
+      e = launch_combine(pb, a.combine, (int)L.cap_combine, part_o, part_lse, stream, false);
     // join (also after an error, so that nothing of the call runs unordered)
     if (ss && ej == cudaSuccess && cudaStreamWaitEvent(stream, ss->join, 0) != cudaSuccess && e == cudaSuccess)
       e = cudaErrorUnknown;

@@ -50,10 +50,24 @@ cudaError_t launch_decode(const Problem &pb, const DecodeItem *items,
                           int n_items, float *partial_o, float *partial_lse,
                           bool pack, cudaStream_t stream);
 
-// Split-KV combine: one warp per (combine item, query head).
+// Split-KV combine: one warp per (combine item, query head).  pdl: queued
+// with programmatic dependent launch right behind the decode launch it
+// merges (its CTAs start during the decode tail and wait on the device).
 cudaError_t launch_combine(const Problem &pb, const CombineItem *items,
                            int n_items, const float *partial_o,
-                           const float *partial_lse, cudaStream_t stream);
+                           const float *partial_lse, cudaStream_t stream, bool pdl);
+
+// Small host-planned decode batches: the work items and combine rows travel
+// in the kernels' launch parameters (host pointers), so no plan copy has to
+// precede the kernels.  pdl: the combine is queued with programmatic
+// dependent launch behind the decode launch.
+bool decode_plan_fits_inline(int n_items, int n_combine);
+cudaError_t launch_decode_inline(const Problem &pb, const DecodeItem *host_items,
+                                 int n_items, float *partial_o, float *partial_lse,
+                                 cudaStream_t stream);
+cudaError_t launch_combine_inline(const Problem &pb, const CombineItem *host_rows,
+                                  int n_items, const float *partial_o,
+                                  const float *partial_lse, cudaStream_t stream, bool pdl);
 
 // Prefill / chunked-prefill kernel (bf16, tcgen05): one CTA per (tile, query
 // head).  head_dim 256: one 128-row tile per CTA.

@@ -192,6 +192,6 @@ extern "C" RPA_API int rpa_decode_noalloc(const void *q, const void *k_new, cons
   pb.causal = 1;
   pb.scale = scale;
   cudaError_t e = launch_decode(pb, d_items, ni, part_o, part_lse, false, stream);
-  if (e == cudaSuccess && nc > 0) e = launch_combine(pb, d_combine, nc, part_o, part_lse, stream);
+  if (e == cudaSuccess && nc > 0) e = launch_combine(pb, d_combine, nc, part_o, part_lse, stream, false);
   return e == cudaSuccess ? RPA_OK : RPA_ERR_CUDA;
 }

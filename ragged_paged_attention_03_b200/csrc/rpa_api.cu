@@ -483,8 +483,9 @@ cudaError_t launch_kernels(DeviceWs &ws, const HostPlan &hp, const int32_t *dev_
     });
   if (L.n_combine > 0 && e == cudaSuccess)
     e = traced(RPA_KERNEL_COMBINE, stream, [&] {
+      // right behind the decode launch unless tracing events sit between them
       return launch_combine(pb, (const CombineItem *)(dev_plan + L.combine_off), (int)L.n_combine, partial_o,
-                            partial_lse, stream);
+                            partial_lse, stream, !g_profile_on.load());
     });
   if (L.n_generic_rows > 0 && e == cudaSuccess)
     e = traced(RPA_KERNEL_GENERIC, stream, [&] {
@@ -622,6 +623,27 @@ extern "C" RPA_API int rpa_forward(const void *q, const void *k_new, const void 
     Slot &slot = ws.slots[ws.next];
     ws.next = (ws.next + 1) % kSlots;
 
+    const PlanLayout &L = hp.layout;
+    if (L.n_prefill_tiles == 0 && L.n_generic_rows == 0 && L.n_decode_packed == 0 && L.n_decode_items > 0 &&
+        decode_plan_fits_inline((int)L.n_decode_items, (int)L.n_combine)) {
+      // A small decode-only batch: its work items and combine rows travel in
+      // the launch parameters, with no plan copy ahead of the kernels.
+      rc = grow_slot(slot, 0, plan_partial_floats(hp, *dims));
+      if (rc) return rc;
+      Problem pb = problem_of(q, k_new, v_new, k_cache, v_cache, page_table, out, lse, *dims, scale, causal);
+      pb.err = ws.err;
+      float *po = slot.partial;
+      float *pl = po ? po + L.n_partials * (int64_t)dims->num_q_heads * dims->head_dim : nullptr;
+      cudaError_t e = traced(RPA_KERNEL_DECODE, stream, [&] {
+        return launch_decode_inline(pb, hp.decode.data(), (int)L.n_decode_items, po, pl, stream);
+      });
+      if (e == cudaSuccess && L.n_combine > 0)
+        e = traced(RPA_KERNEL_COMBINE, stream, [&] {
+          return launch_combine_inline(pb, hp.combine.data(), (int)L.n_combine, po, pl, stream, !g_profile_on.load());
+        });
+      if (cudaEventRecord(slot.done, stream) == cudaSuccess) slot.pending = true;
+      return e == cudaSuccess ? RPA_OK : RPA_ERR_CUDA;
+    }
     rc = grow_slot(slot, hp.layout.total_words, plan_partial_floats(hp, *dims));
     if (rc) return rc;
     serialize(hp, slot.host);
