@@ -526,8 +526,9 @@ def main():
                     help="replicas: every GPU runs the whole batch (weak scaling); heads: every GPU "
                          "runs its Hkv/N KV heads of the same batch (strong scaling; no collective)")
     ap.add_argument("--prefill-kernel", type=int, default=None,
-                    help="RPA_OPT_PREFILL_KERNEL for the head_dim 128 prefill (0 or 1: two tiles per CTA, "
-                         "the default; 2: CTA pairs; 3: one tile per CTA)")
+                    help="RPA_OPT_PREFILL_KERNEL (0, the default: two tiles per CTA at head_dim 128, CTA "
+                         "pairs at 256; 1: two tiles per CTA, one tile per CTA at 256; 2: CTA pairs; 3: one "
+                         "tile per CTA at 128)")
     ap.add_argument("--ablate-write", action="store_true",
                     help="time each workload's kernels with and without the fused cache stores "
                          "(a separate timing-only build; off by default)")

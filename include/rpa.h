@@ -216,15 +216,19 @@ enum {
                                       (two per SM); fewer stay in the main
                                       decode launch (default 64; 0 restores
                                       it, < 0: never) */
-  RPA_OPT_PREFILL_KERNEL = 7       /* head_dim 128 prefill kernel: 0 (default)
-                                      or 1 two 128-row tiles per CTA (the
-                                      head_dim 64 kernel); 2 CTA pairs
-                                      sharing M = 256 tcgen05 MMAs, one
-                                      256-row item per pair, three score
-                                      buffers; 3 the same with one 128-row
-                                      tile per CTA.  Results agree within
-                                      rounding; 2 and 3 measured slower and
-                                      are kept for measurement */
+  RPA_OPT_PREFILL_KERNEL = 7       /* prefill kernel.  0 (default): the
+                                      head_dim 64 / 128 kernel with two
+                                      128-row tiles per CTA, and CTA pairs
+                                      sharing M = 256 tcgen05 MMAs at
+                                      head_dim 256 (one 256-row item per
+                                      pair); 1: the two-tile kernel, and one
+                                      128-row tile per CTA at head_dim 256;
+                                      2: CTA pairs at head_dim 128 and 256;
+                                      3: the head_dim 128 pair design on one
+                                      CTA per 128-row tile.  Results agree
+                                      within rounding.  The device workspace
+                                      size depends on it at head_dim 256
+                                      (item rows) */
 };
 RPA_API int64_t rpa_set_option(int32_t option, int64_t value);
 
@@ -300,7 +304,8 @@ RPA_API int rpa_decode_noalloc(const void *q, const void *k_new,
  * needs for batches of at most max_seqs sequences under dims (total_q_tokens
  * is the row capacity T of q / k_new / v_new / out).  It depends on dims,
  * max_seqs and the current RPA_OPT_DECODE_CHUNK_BLOCKS and
- * RPA_OPT_DECODE_PACK_BLOCKS values only.  Host only; returns RPA_OK or the
+ * RPA_OPT_DECODE_PACK_BLOCKS values (and, at head_dim 256,
+ * RPA_OPT_PREFILL_KERNEL) only.  Host only; returns RPA_OK or the
  * RPA_ERR_* code of bad dims / max_seqs < 0 (then *bytes = 0).
  */
 RPA_API int rpa_device_workspace_size(const rpa_dims *dims, int32_t max_seqs,

@@ -91,6 +91,8 @@ cudaError_t launch_prefill3(const Problem &pb, const PrefillTile *tiles,
 constexpr int kPrefillTileRows = 128;
 
 // Rows of one prefill work item for a head dim.
-inline int prefill_item_rows(int head_dim) { return head_dim <= 128 ? 256 : 128; }
+// head_dim <= 128: 256 (two tiles, or a CTA pair); head_dim 256: 256 (a CTA
+// pair), or 128 when RPA_OPT_PREFILL_KERNEL selects the one-tile kernel.
+int prefill_item_rows(int head_dim);
 
 }  // namespace rpa

@@ -64,30 +64,40 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O when the max grows by > 2^8
 
-template <bool PAIR>
+template <bool PAIR, int HEAD_DIM>
 struct P3 {
-  static constexpr int D = 128;
+  static constexpr int D = HEAD_DIM;
   static constexpr int BM = 128;                 // query rows per CTA
   static constexpr int BN = 128;                 // keys per block
   static constexpr int NCTA = PAIR ? 2 : 1;
   static constexpr int KH = BN / NCTA;           // keys of each K block this CTA holds
   static constexpr int VC = D / NCTA;            // head-dim columns of each V block this CTA holds
   static constexpr int VH = VC / 64;             // 128-byte column slabs of a V block
-  static constexpr int kQBytes = BM * D * 2;     // 32 KB
-  static constexpr int kKBytes = KH * D * 2;     // 16 KB (pair) / 32 KB
-  static constexpr int kVBytes = BN * VC * 2;    // 16 KB (pair) / 32 KB
-  static constexpr int NSK = PAIR ? 4 : 2;
-  static constexpr int NSV = PAIR ? 4 : 2;
-  static constexpr int kData = 2 * kQBytes + NSK * kKBytes + NSV * kVBytes;
+  static constexpr int kQBytes = BM * D * 2;     // 32 KB (head_dim 128) / 64 KB (256)
+  static constexpr int kKBytes = KH * D * 2;
+  static constexpr int kVBytes = BN * VC * 2;
+  // head_dim 128: two Q buffers (the next unit's Q loads during this one)
+  // and deep K/V rings; head_dim 256 (pairs only): one Q buffer and two
+  // stages each of half-blocks, 192 KB in all
+  static constexpr int NQ = D == 128 ? 2 : 1;
+  static constexpr int NSK = D == 128 ? (PAIR ? 4 : 2) : 2;
+  static constexpr int NSV = D == 128 ? (PAIR ? 4 : 2) : 2;
+  static constexpr int kData = NQ * kQBytes + NSK * kKBytes + NSV * kVBytes;
   static constexpr int HK = BN / 2;               // keys of a block per softmax warpgroup
   static constexpr int kStatFloats = 2 * 3 * BM;   // [unit parity][l of keys 0-63, l of keys 64-127, m][row]
   static constexpr int kRedFloats = 2 * 2 * BM;    // [exchange parity][warpgroup][row]: partial row maxima
   static constexpr int kSmem = 1024 + kData + (kStatFloats + kRedFloats) * 4 + 512;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr int NS = 3;                    // S buffers: S(i) at i * 128
-  static constexpr uint32_t kColO = 384;          // O
+  // TMEM: NS score buffers of 128 columns, then O (D columns): three score
+  // buffers at head_dim 128, two at 256
+  static constexpr int NS = D == 128 ? 3 : 2;
+  static constexpr uint32_t kColO = NS * 128;
+  static constexpr int kLag = NS - 1;             // PV(b - kLag) is issued after QK(b)
   static constexpr uint32_t kSoftmaxArrivals = 8 * NCTA;   // one elected lane per softmax warp, per CTA
   static constexpr uint32_t kEpilogueArrivals = 4 * NCTA;  // one per epilogue warp, per CTA
+  static_assert(kColO + D <= kTmemCols, "TMEM columns");
+  static_assert(kSmem <= 232448, "shared memory per CTA");
+  static_assert(PAIR || D == 128, "head_dim 256 runs on CTA pairs only");
 };
 
 struct Bars3 {
@@ -192,7 +202,7 @@ struct Unit3 {
 template <bool PAIR>
 __device__ __forceinline__ Unit3 make_unit3(const PrefillTile *tiles, int u, int n_units, const Problem &pb,
                                             int rank) {
-  using S = P3<PAIR>;
+  using S = P3<PAIR, 128>;   // rows and keys per block do not depend on D
   Unit3 w{};
   w.end = u >= n_units;
   if (w.end) return w;
@@ -218,9 +228,9 @@ __device__ __forceinline__ Unit3 make_unit3(const PrefillTile *tiles, int u, int
 }
 
 // ---------------------------------------------------------------- MMA
-template <bool PAIR>
+template <bool PAIR, int D>
 __device__ __forceinline__ void mma_qk(uint32_t tS, uint64_t dq, uint64_t dk) {
-  using S = P3<PAIR>;
+  using S = P3<PAIR, D>;
   constexpr uint32_t idesc = ptx::umma_idesc_bf16(PAIR ? 256 : 128, S::BN, false);
 #pragma unroll
   for (int ks = 0; ks < S::D / 16; ++ks) {
@@ -233,9 +243,9 @@ __device__ __forceinline__ void mma_qk(uint32_t tS, uint64_t dq, uint64_t dk) {
   }
 }
 
-template <bool PAIR>
+template <bool PAIR, int D>
 __device__ __forceinline__ void mma_pv(uint32_t tO, uint32_t tP, uint64_t dv, bool first) {
-  using S = P3<PAIR>;
+  using S = P3<PAIR, D>;
   constexpr uint32_t idesc = ptx::umma_idesc_bf16(PAIR ? 256 : 128, S::D, true);
 #pragma unroll
   for (int kk = 0; kk < S::BN / 16; ++kk) {
@@ -261,9 +271,9 @@ struct PendingPV {
   bool first, last;
 };
 
-template <bool PAIR>
+template <bool PAIR, int D>
 __device__ __forceinline__ bool issue_pending_pv(const Sync &sy, const PendingPV &pv, uint32_t tmem, uint64_t dv0) {
-  using S = P3<PAIR>;
+  using S = P3<PAIR, D>;
   Bars3 *bars = sy.bars;
   const int sb = pv.gb % S::NS;
   if (!wait_all3<PAIR>(sy, &bars->p_full[sb], (uint32_t)((pv.gb / S::NS) & 1))) return false;
@@ -273,46 +283,51 @@ __device__ __forceinline__ bool issue_pending_pv(const Sync &sy, const PendingPV
   // have read it
   if (pv.first && pv.gu >= 1 && !wait_all3<PAIR>(sy, &bars->o_free, (uint32_t)((pv.gu - 1) & 1))) return false;
   ptx::tc_fence_after();
-  mma_pv<PAIR>(tmem + S::kColO, tmem + sb * 128, dv0 + (uint64_t)((vs * S::kVBytes) >> 4), pv.first);
+  mma_pv<PAIR, D>(tmem + S::kColO, tmem + sb * 128, dv0 + (uint64_t)((vs * S::kVBytes) >> 4), pv.first);
   commit<PAIR>(&bars->v_empty[vs]);
   commit<PAIR>(&bars->pv_done[pv.gb & 1]);
   if (pv.last) commit<PAIR>(&bars->o_full);
   return true;
 }
 
-template <bool PAIR>
+template <bool PAIR, int D>
 __device__ __forceinline__ void mma_loop(const Sync &sy, const Problem &pb, const PrefillTile *tiles, int n_units,
                                          uint32_t tmem, uint32_t q_addr, uint32_t k_addr, uint32_t v_addr) {
-  using S = P3<PAIR>;
+  using S = P3<PAIR, D>;
   Bars3 *bars = sy.bars;
   const uint64_t dq0 = ptx::umma_desc_sw128(q_addr, 16, 1024);
   const uint64_t dk0 = ptx::umma_desc_sw128(k_addr, 16, 1024);
   const uint64_t dv0 = ptx::umma_desc_sw128(v_addr, S::BN * 128, 1024);
   int gb = 0, gu = 0;
   bool ok = true;
-  int npend = 0;          // PVs queued behind the QKs (at most two: pa, then pb)
+  int npend = 0;          // PVs queued behind the QKs (at most kLag: pa, then pbv)
   PendingPV pa{}, pbv{};
   for (int k = 0; ok; ++k) {
     const Unit3 w = make_unit3<PAIR>(tiles, unit_of<PAIR>(k), n_units, pb, 0);
     if (w.end) break;
     if (w.skip) continue;
-    const int qb = gu & 1;
-    ok = wait_all3<PAIR>(sy, &bars->q_full[qb], (uint32_t)((gu >> 1) & 1));
+    const int qb = gu % S::NQ;
+    ok = wait_all3<PAIR>(sy, &bars->q_full[qb], (uint32_t)((gu / S::NQ) & 1));
     for (int j = 0; ok && j < w.nb; ++j, ++gb) {
       const int ks = gb % S::NSK;
       ok = wait_all3<PAIR>(sy, &bars->k_full[ks], (uint32_t)((gb / S::NSK) & 1));
       if (!ok) break;
       ptx::tc_fence_after();
-      mma_qk<PAIR>(tmem + (gb % S::NS) * 128, dq0 + (uint64_t)((qb * S::kQBytes) >> 4),
+      mma_qk<PAIR, D>(tmem + (gb % S::NS) * 128, dq0 + (uint64_t)((qb * S::kQBytes) >> 4),
                    dk0 + (uint64_t)((ks * S::kKBytes) >> 4));
       commit<PAIR>(&bars->k_empty[ks]);
       commit<PAIR>(&bars->s_full[gb % S::NS]);
       if (j + 1 == w.nb) commit<PAIR>(&bars->q_empty[qb]);
+      // queue PV(gb); issue PV(gb - kLag) now
       const PendingPV cur{gb, gu, j == 0, j + 1 == w.nb};
-      if (npend == 2) {
-        ok = issue_pending_pv<PAIR>(sy, pa, tmem, dv0);
-        pa = pbv;
-        pbv = cur;
+      if (npend == S::kLag) {
+        ok = issue_pending_pv<PAIR, D>(sy, pa, tmem, dv0);
+        if (S::kLag == 2) {
+          pa = pbv;
+          pbv = cur;
+        } else {
+          pa = cur;
+        }
       } else if (npend == 1) {
         pbv = cur;
         npend = 2;
@@ -323,8 +338,8 @@ __device__ __forceinline__ void mma_loop(const Sync &sy, const Problem &pb, cons
     }
     ++gu;
   }
-  if (ok && npend >= 1) ok = issue_pending_pv<PAIR>(sy, pa, tmem, dv0);
-  if (ok && npend == 2) issue_pending_pv<PAIR>(sy, pbv, tmem, dv0);
+  if (ok && npend >= 1) ok = issue_pending_pv<PAIR, D>(sy, pa, tmem, dv0);
+  if (ok && npend == 2) issue_pending_pv<PAIR, D>(sy, pbv, tmem, dv0);
 }
 
 // ------------------------------------------------------------ producer
@@ -444,11 +459,11 @@ __device__ __forceinline__ bool load_block(const Sync &sy, const Problem &pb, co
 
 // One producer warp per operand: IS_V loads V, otherwise Q and K.  Each
 // fills its own stage ring as soon as the MMA warp releases a stage.
-template <bool PAIR, bool IS_V>
+template <bool PAIR, bool IS_V, int D>
 __device__ __forceinline__ void produce(const Sync &sy, const Problem &pb, const PrefillTile *tiles, int n_units,
                                         int rank, uint8_t *sQ, uint8_t *sOp, const CUtensorMap *tm_q,
                                         const CUtensorMap *tm_ctx, const CUtensorMap *tm_new) {
-  using S = P3<PAIR>;
+  using S = P3<PAIR, D>;
   constexpr int NS = IS_V ? S::NSV : S::NSK;
   Bars3 *bars = sy.bars;
   uint64_t *full = IS_V ? bars->v_full : bars->k_full;
@@ -465,9 +480,10 @@ __device__ __forceinline__ void produce(const Sync &sy, const Problem &pb, const
     if (w.skip) continue;
     const int32_t *pt_row = pb.page_table + (size_t)w.tile.seq * pb.max_pages;
     if (!IS_V) {
-      // Q of this CTA's rows, once the unit two back has finished its QKs
-      const int qb = gu & 1;
-      if (gu >= 2 && !wait_all3<PAIR>(sy, &bars->q_empty[qb], (uint32_t)(((gu - 2) >> 1) & 1))) break;
+      // Q of this CTA's rows, once the unit that last used the buffer has
+      // finished its QKs
+      const int qb = gu % S::NQ;
+      if (gu >= S::NQ && !wait_all3<PAIR>(sy, &bars->q_empty[qb], (uint32_t)(((gu - S::NQ) / S::NQ) & 1))) break;
       const uint32_t qbar = leader_bar<PAIR>(&bars->q_full[qb]);
       if (lane == 0) {
         if constexpr (PAIR)
@@ -476,12 +492,15 @@ __device__ __forceinline__ void produce(const Sync &sy, const Problem &pb, const
           ptx::mbar_arrive_expect_tx(&bars->q_full[qb], S::kQBytes);
       }
       __syncwarp();
+      // Q is read once: first out of L2, ahead of the K/V blocks that the
+      // other query heads and later items of the sequence read again
+      const uint64_t once = ptx::l2_evict_first_policy();
       for (int hh = 0; hh < S::D / 64; ++hh) {
         uint8_t *d = sQ + qb * S::kQBytes + hh * S::BM * 128;
         if constexpr (PAIR)
-          ptx::tma_load_3d_pair_elect(d, tm_q, qbar, hh * 64, w.h, w.tile.q_start + w.my_r0);
+          ptx::tma_load_3d_pair_hint_elect(d, tm_q, qbar, hh * 64, w.h, w.tile.q_start + w.my_r0, once);
         else
-          ptx::tma_load_3d_elect(d, tm_q, &bars->q_full[qb], hh * 64, w.h, w.tile.q_start + w.my_r0);
+          ptx::tma_load_3d_hint_elect(d, tm_q, &bars->q_full[qb], hh * 64, w.h, w.tile.q_start + w.my_r0, once);
       }
     }
     for (int j = 0; j < w.nb; ++j, ++gb) {
@@ -517,9 +536,9 @@ __device__ __forceinline__ void produce(const Sync &sy, const Problem &pb, const
 // their page slots: the G query heads of a KV head split the unit's rows,
 // and the two CTAs of a pair split each share.  Each lane keeps kBatch
 // 16-byte chunks (and their page-table entries) in flight before storing.
-template <bool PAIR>
+template <bool PAIR, int D>
 __device__ __forceinline__ void cache_update(const Problem &pb, const PrefillTile *tiles, int n_units, int rank) {
-  using S = P3<PAIR>;
+  using S = P3<PAIR, D>;
   if (!kCacheWrite) return;
   constexpr int kBatch = 8;
   const int lane = threadIdx.x & 31;
@@ -588,11 +607,11 @@ __device__ __forceinline__ void cache_update(const Problem &pb, const PrefillTil
 // reference max moves only when a block's max exceeds it by more than 2^8 (a
 // lazy rescale, exact after the final 1 / l); O is then rescaled once
 // PV(b - 1) is complete.
-template <bool PAIR>
+template <bool PAIR, int D>
 __device__ __forceinline__ void softmax_loop(const Sync &sy, const Problem &pb, const PrefillTile *tiles,
                                              int n_units, int rank, uint32_t tmem, float *stats, float *red,
                                              float scale_log2) {
-  using S = P3<PAIR>;
+  using S = P3<PAIR, D>;
   constexpr int BN = S::BN, HK = S::HK;
   Bars3 *bars = sy.bars;
   const int warp = threadIdx.x >> 5;
@@ -600,7 +619,7 @@ __device__ __forceinline__ void softmax_loop(const Sync &sy, const Problem &pb, 
   const int wq = warp & 3;                           // warp of the pair (rows 32 wq ..)
   const int row = threadIdx.x & 127;                 // TMEM lane
   const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
-  const uint32_t tO = lane_base + S::kColO + (uint32_t)(half * HK);
+  const uint32_t tO = lane_base + S::kColO + (uint32_t)(half * (S::D / 2));   // this warpgroup's half of O
   int gb = 0, gu = 0;
   int xc = 0;   // exchanges of this warp pair so far (blocks it skips have none)
   bool ok = true;
@@ -684,7 +703,7 @@ __device__ __forceinline__ void softmax_loop(const Sync &sy, const Problem &pb, 
             }
             ptx::tc_fence_after();
 #pragma unroll 1
-            for (int cc = 0; cc < HK / 32; ++cc) {
+            for (int cc = 0; cc < S::D / 64; ++cc) {
               uint32_t r[32];
               ptx::tmem_ld32(tO + cc * 32, r);
               ptx::tmem_ld_wait();
@@ -737,10 +756,10 @@ __device__ __forceinline__ void softmax_loop(const Sync &sy, const Problem &pb, 
 }
 
 // ------------------------------------------------------------- epilogue
-template <bool PAIR>
+template <bool PAIR, int D>
 __device__ __forceinline__ void epilogue_loop(const Sync &sy, const Problem &pb, const PrefillTile *tiles,
                                               int n_units, int rank, uint32_t tmem, const float *stats) {
-  using S = P3<PAIR>;
+  using S = P3<PAIR, D>;
   Bars3 *bars = sy.bars;
   const int warp = threadIdx.x >> 5;
   const int row = threadIdx.x & 127;
@@ -764,6 +783,7 @@ __device__ __forceinline__ void epilogue_loop(const Sync &sy, const Problem &pb,
     const bool store = row < w.my_rows;
     const int rn = w.my_r0 + row;
     const float inv = store ? 1.f / l : 0.f;
+    const uint64_t once = ptx::l2_evict_first_policy();   // outputs are written once: first out of L2
     uint4 *out = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(pb.out) +
                                            ((size_t)(w.tile.q_start + (store ? rn : 0)) * pb.hq + w.h) * S::D);
 #pragma unroll 1
@@ -778,7 +798,7 @@ __device__ __forceinline__ void epilogue_loop(const Sync &sy, const Problem &pb,
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             o2[i] = ptx::pack_bf16(__uint_as_float(ov[q * 8 + 2 * i]) * inv, __uint_as_float(ov[q * 8 + 2 * i + 1]) * inv);
-          out[cc * 4 + q] = make_uint4(o2[0], o2[1], o2[2], o2[3]);
+          ptx::st_global_hint(out + cc * 4 + q, make_uint4(o2[0], o2[1], o2[2], o2[3]), once);
         }
       }
     }
@@ -790,17 +810,17 @@ __device__ __forceinline__ void epilogue_loop(const Sync &sy, const Problem &pb,
 }
 
 // --------------------------------------------------------------- kernel
-template <bool PAIR>
+template <bool PAIR, int D>
 __global__ void __launch_bounds__(512, 1)
     prefill3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
                     const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_kn,
                     const __grid_constant__ CUtensorMap tm_vn, const Problem pb,
                     const PrefillTile *__restrict__ tiles, int n_units, float scale_log2) {
-  using S = P3<PAIR>;
+  using S = P3<PAIR, D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sQ = base;                     // Q buffer b at sQ + b * kQBytes
-  uint8_t *sK = sQ + 2 * S::kQBytes;
+  uint8_t *sK = sQ + S::NQ * S::kQBytes;
   uint8_t *sV = sK + S::NSK * S::kKBytes;
   float *stats = reinterpret_cast<float *>(base + S::kData);
   float *red = stats + S::kStatFloats;
@@ -878,12 +898,12 @@ __global__ void __launch_bounds__(512, 1)
 
   if (warp >= 12) {
     if (warp == 12) {
-      produce<PAIR, false>(sy, pb, tiles, n_units, rank, sQ, sK, &tm_q, &tm_kc, &tm_kn);
+      produce<PAIR, false, D>(sy, pb, tiles, n_units, rank, sQ, sK, &tm_q, &tm_kc, &tm_kn);
     } else if (warp == 14) {
-      produce<PAIR, true>(sy, pb, tiles, n_units, rank, sQ, sV, &tm_q, &tm_vc, &tm_vn);
+      produce<PAIR, true, D>(sy, pb, tiles, n_units, rank, sQ, sV, &tm_q, &tm_vc, &tm_vn);
     } else if (warp == 13) {
       if (rank == 0) {
-        mma_loop<PAIR>(sy, pb, tiles, n_units, tmem, ptx::smem_u32(sQ), ptx::smem_u32(sK), ptx::smem_u32(sV));
+        mma_loop<PAIR, D>(sy, pb, tiles, n_units, tmem, ptx::smem_u32(sQ), ptx::smem_u32(sK), ptx::smem_u32(sV));
         // every MMA this warp issued is complete before the CTA (and, through
         // the exit handshake below, its peer) releases TMEM or leaves
         commit<PAIR>(&bars->drain);
@@ -891,12 +911,12 @@ __global__ void __launch_bounds__(512, 1)
         __syncwarp();
       }
     } else {
-      cache_update<PAIR>(pb, tiles, n_units, rank);
+      cache_update<PAIR, D>(pb, tiles, n_units, rank);
     }
   } else if (warp < 8) {
-    softmax_loop<PAIR>(sy, pb, tiles, n_units, rank, tmem, stats, red, scale_log2);
+    softmax_loop<PAIR, D>(sy, pb, tiles, n_units, rank, tmem, stats, red, scale_log2);
   } else {
-    epilogue_loop<PAIR>(sy, pb, tiles, n_units, rank, tmem, stats);
+    epilogue_loop<PAIR, D>(sy, pb, tiles, n_units, rank, tmem, stats);
   }
 
   ptx::tc_fence_before();
@@ -919,9 +939,9 @@ __global__ void __launch_bounds__(512, 1)
   }
 }
 
-template <bool PAIR>
+template <bool PAIR, int D>
 cudaError_t launch_t(const Problem &pb, const PrefillTile *tiles, int n_tiles, int max_ctas, cudaStream_t stream) {
-  using S = P3<PAIR>;
+  using S = P3<PAIR, D>;
   CUtensorMap tq, tkc, tvc, tkn, tvn;
   const uint64_t qdims[3] = {(uint64_t)S::D, (uint64_t)pb.hq, (uint64_t)pb.total_q};
   const uint64_t qstr[2] = {(uint64_t)S::D * 2, (uint64_t)pb.hq * S::D * 2};
@@ -940,7 +960,7 @@ cudaError_t launch_t(const Problem &pb, const PrefillTile *tiles, int n_tiles, i
       !make_tmap_bf16_3d(&tkn, pb.k_new, ndims, nstr, knbox, true) ||
       !make_tmap_bf16_3d(&tvn, pb.v_new, ndims, nstr, vnbox, true))
     return cudaErrorInvalidValue;
-  auto kern = prefill3_kernel<PAIR>;
+  auto kern = prefill3_kernel<PAIR, D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem);
   if (e != cudaSuccess) return e;
   const int n_units = n_tiles * (PAIR ? pb.hq : 2 * pb.hq);
@@ -1001,9 +1021,11 @@ cudaError_t launch_t(const Problem &pb, const PrefillTile *tiles, int n_tiles, i
 cudaError_t launch_prefill3(const Problem &pb, const PrefillTile *tiles, int n_tiles, int max_ctas, bool pair,
                             cudaStream_t stream) {
   if (n_tiles <= 0) return cudaSuccess;
-  if (pb.d != 128) return cudaErrorInvalidValue;
-  return pair ? launch_t<true>(pb, tiles, n_tiles, max_ctas, stream)
-              : launch_t<false>(pb, tiles, n_tiles, max_ctas, stream);
+  if (pb.d == 128)
+    return pair ? launch_t<true, 128>(pb, tiles, n_tiles, max_ctas, stream)
+                : launch_t<false, 128>(pb, tiles, n_tiles, max_ctas, stream);
+  if (pb.d == 256 && pair) return launch_t<true, 256>(pb, tiles, n_tiles, max_ctas, stream);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace rpa

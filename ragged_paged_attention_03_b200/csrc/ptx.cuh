@@ -390,6 +390,17 @@ __device__ __forceinline__ void tma_load_3d_pair_elect(void *dst, const void *tm
       : "memory");
 }
 
+// The same, with an L2 cache policy (e.g. evict-first for data read once).
+__device__ __forceinline__ void tma_load_3d_pair_hint_elect(void *dst, const void *tmap, uint32_t bar_cluster,
+                                                            int32_t c0, int32_t c1, int32_t c2, uint64_t policy) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1, {%3, %4, %5}], [%2], %6;\n\t}" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
+      : "memory");
+}
+
 // TMEM allocation shared by the pair: the warp with the same index in both
 // CTAs executes it; each CTA gets the same columns of its own TMEM.
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst, uint32_t ncols) {

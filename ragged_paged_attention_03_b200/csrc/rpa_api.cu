@@ -68,10 +68,18 @@ int64_t prefill_sms() { return g_opt_prefill_sms.load(); }
 
 int64_t prefill_kernel() { return g_opt_prefill_kernel.load(); }
 
+int prefill_item_rows(int head_dim) {
+  if (head_dim <= 128) return 256;
+  return prefill_kernel() == 1 ? 128 : 256;
+}
+
 cudaError_t launch_prefill_any(const Problem &pb, const PrefillTile *tiles, int n_tiles, int max_ctas, bool split,
                                cudaStream_t stream) {
-  if (pb.d == 256) return launch_prefill(pb, tiles, n_tiles, stream);
   const int64_t k = prefill_kernel();
+  // head_dim 256: CTA pairs unless the one-tile kernel is asked for (its
+  // items are 128 rows; prefill_item_rows follows the same choice)
+  if (pb.d == 256) return k == 1 ? launch_prefill(pb, tiles, n_tiles, stream)
+                                 : launch_prefill3(pb, tiles, n_tiles, max_ctas, true, stream);
   if (pb.d == 128 && (k == 2 || k == 3)) return launch_prefill3(pb, tiles, n_tiles, max_ctas, k == 2, stream);
   return launch_prefill2(pb, tiles, n_tiles, max_ctas, split, stream);
 }

@@ -1,11 +1,11 @@
-"""The head_dim-128 prefill kernel built on CTA pairs (tcgen05 MMAs of
-M = 256 across two SMs, three score buffers, a separate epilogue warpgroup)
-and its one-CTA form, forced through RPA_OPT_PREFILL_KERNEL, against the
-fp64 oracle: every output row and the whole cache pool on small mixes
-(fresh and chunked prefill with ragged tails, page sizes 8 to 256, causal
-and not), and sampled rows plus whole-pool cache properties on the full-size
-causal prefill batch.  Neither form is the default kernel; both must agree
-with the oracle all the same.
+"""Prefill kernels other than each head dim's default, forced through
+RPA_OPT_PREFILL_KERNEL, against the fp64 oracle: the CTA-pair kernel (tcgen05
+MMAs of M = 256 across two SMs, a separate epilogue warpgroup; the default at
+head_dim 256) at head_dim 128 and its one-CTA form, and the one-tile-per-CTA
+head_dim-256 kernel.  Every output row and the whole cache pool on small
+mixes (fresh and chunked prefill with ragged tails, page sizes 8 to 256,
+causal and not), and sampled rows plus whole-pool cache properties on a
+full-size causal prefill batch of each head dim.
 """
 import numpy as np
 import pytest
@@ -19,7 +19,9 @@ from test_parity_gpu import SMALL, MORE, full_check, sampled_check
 pytestmark = pytest.mark.gpu
 
 KERNELS = {2: "pair", 3: "single"}
+# head_dim 256: the pair kernel is the default; the one-tile kernel is forced with 1
 CASES = [("small", i) for i in (0, 4, 5, 6, 7, 10)] + [("more", i) for i in (1, 2)]
+CASES_256 = [("small", 9), ("more", 3), ("more", 4)]   # head_dim 256: pairs only
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -49,9 +51,21 @@ def test_forced_prefill_kernel(oracle_mod, kernel_option, table, case):
     full_check(oracle_mod, prob)
 
 
-@pytest.mark.parametrize("kernel_option", [2], ids=["pair"], indirect=True)
-def test_forced_pair_full_causal_prefill(oracle_mod, kernel_option):
-    prob = I.make_workload("prefill_8x2048", device="cuda")
+@pytest.mark.parametrize("kernel_option", [2, 1], ids=["pair", "one-tile"], indirect=True)
+@pytest.mark.parametrize("table,case", CASES_256, ids=[f"{t}{c}" for t, c in CASES_256])
+def test_forced_head_dim_256(oracle_mod, kernel_option, table, case):
+    ql, kv, hq, hkv, d, p, causal = (SMALL if table == "small" else MORE)[case]
+    assert d == 256
+    seed, pool = (100 + case, 1.5) if table == "small" else (500 + case, 1.3)
+    prob = I.make_problem(ql, kv, num_q_heads=hq, num_kv_heads=hkv, head_dim=d, page_size=p,
+                          dtype=I.BF16, causal=causal, seed=seed, pool=pool)
+    full_check(oracle_mod, prob)
+
+
+@pytest.mark.parametrize("kernel_option,name", [(2, "prefill_8x2048"), (1, "prefill_4x4096_d256")],
+                         ids=["pair-d128", "one-tile-d256"], indirect=["kernel_option"])
+def test_forced_full_causal_prefill(oracle_mod, kernel_option, name):
+    prob = I.make_workload(name, device="cuda")
     pre_k, pre_v = prob.k_cache.clone(), prob.v_cache.clone()
     from harness import run_gpu
     out, lse, flags = run_gpu(prob)
