@@ -100,6 +100,9 @@ def peaks():
         return dict(hbm=6650.0, tc=1590.0, tc_sustained=1400.0, source="fallback")
 
 
+PREFILL_KERNEL_OPTION = 0   # RPA_OPT_PREFILL_KERNEL of this run (--prefill-kernel)
+
+
 def traffic_for(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if the kernel's
     source has not changed since those counters were taken."""
@@ -110,6 +113,9 @@ def traffic_for(kernel: str, workload: str):
     except (OSError, ValueError):
         return None
     if not rec:
+        return None
+    # the counters belong to the kernel that the RPA_OPT_PREFILL_KERNEL of the capture picks
+    if PREFILL_KERNEL_OPTION != rec.get("prefill_kernel_option", 0):
         return None
     src = os.path.join(ROOT, rec["source"])
     try:
@@ -473,8 +479,9 @@ def ablate_write(args, dev):
     for spec in [w for w in args.workloads.split(",") if w]:
         with_w, step_w = kernel_times(spec, args.steps, args.warmup, dev)
         env = dict(os.environ, RPA_ABLATE_CACHE_WRITE="1")
+        kopt = [] if args.prefill_kernel is None else ["--prefill-kernel", str(args.prefill_kernel)]
         r = subprocess.run([sys.executable, os.path.abspath(__file__), "--ablate-child", "--workloads", spec,
-                            "--steps", str(args.steps), "--warmup", str(args.warmup)],
+                            "--steps", str(args.steps), "--warmup", str(args.warmup)] + kopt,
                            env=env, capture_output=True, text=True, check=True)
         child = json.loads(r.stdout.strip().splitlines()[-1])
         without, step_wo = child["kern"], child["ms_per_step"]
@@ -534,6 +541,11 @@ def main():
                          "(a separate timing-only build; off by default)")
     ap.add_argument("--ablate-child", action="store_true", help=argparse.SUPPRESS)
     args = ap.parse_args()
+    if args.prefill_kernel is not None:
+        global PREFILL_KERNEL_OPTION
+        from ragged_paged_attention_03_b200 import binding as rb
+        rb.rpa_set_option(rb.RPA_OPT_PREFILL_KERNEL, args.prefill_kernel)
+        PREFILL_KERNEL_OPTION = args.prefill_kernel
     if args.ablate_write or args.ablate_child:
         dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
         torch.cuda.set_device(dev)
@@ -547,9 +559,6 @@ def main():
         return
     world, rank, local = dist_setup(args)
     n = world
-    if args.prefill_kernel is not None:
-        from ragged_paged_attention_03_b200 import binding as rb
-        rb.rpa_set_option(rb.RPA_OPT_PREFILL_KERNEL, args.prefill_kernel)
     wl = [w for w in args.workloads.split(",") if w]
 
     if args.impl == "reference":

@@ -1,9 +1,12 @@
-// prefill3_kernel.cu -- prefill / chunked-prefill attention for head_dim 128
-// with a double-buffered score tile: while the softmax warps turn S(j) into
-// P(j), the tensor cores compute S(j+1) = Q K(j+1)^T and O += P(j-1) V(j-1),
-// so a block costs the larger of the softmax time and the MMA time instead
-// of their sum (the compute-bound prefill regime of the RPA talk summary,
-// 00:11:09; the cache update of 00:06:36 is fused here too).
+// prefill3_kernel.cu -- prefill / chunked-prefill attention with score
+// tiles computed ahead of the softmax: while the softmax warps turn S(j) into
+// P(j), the tensor cores compute the next block's S = Q K^T and an earlier
+// block's O += P V, so a block costs the larger of the softmax time and the
+// MMA time instead of their sum (the compute-bound prefill regime of the RPA
+// talk summary, 00:11:09; the cache update of 00:06:36 is fused here too).
+// It is the default prefill kernel at head_dim 256, where the MMA work of a
+// block (QK at N = 128 plus PV at N = 256) outweighs its softmax; at head_dim
+// 128 it is selectable (the two-tile kernel in prefill2_kernel.cu is faster).
 //
 // Two builds of one kernel:
 //  * PAIR = true: a cluster of two CTAs on two SMs works on one 256-row work
@@ -30,25 +33,28 @@
 //               keys (context from cache pages, new tokens from k_new; rows
 //               without a valid key zeroed)
 //   warp 13     TMEM allocation; MMA issue (the leader's, in a pair)
-//   warp 14     TMA producer of V blocks (as for K): V(b) waits for PV(b - 4),
-//               which is queued two blocks behind QK(b - 2), so a producer
-//               shared with K would hold every K load back by as much
+//   warp 14     TMA producer of V blocks (as for K): V(b) waits for the PV
+//               that last read its stage (PV(b - 4) at head_dim 128), which
+//               is queued NS - 1 blocks behind its QK, so a producer shared
+//               with K would hold every K load back by as much
 //   warp 15     fused cache update: this CTA's share of the unit's new K/V
 //               rows copied into their page slots
 //
 // TMEM (512 columns, the same columns in both CTAs of a pair):
-//   S(0) | S(1) | S(2) | O, 128 columns each.  Blocks cycle through the three
-//   S buffers; O holds one unit at a time.
+//   head_dim 128: S(0) | S(1) | S(2) | O, 128 columns each (NS = 3);
+//   head_dim 256: S(0) | S(1) | O, with O 256 columns wide (NS = 2).
+//   Blocks cycle through the NS score buffers; O holds one unit at a time.
 //
 // The MMA warp issues, per block b (counted over all units of the CTA):
-//   QK(b) into S(b mod 3), then PV(b - 2) from P(b - 2).  QK(b) therefore
-//   waits for no softmax: the buffer it overwrites was last read by PV(b - 3),
-//   issued before it, and tcgen05 operations issued by one thread execute in
-//   order.  While the softmax warps turn S(b) into P(b), S(b + 1) is already
-//   computed and S(b + 2) is being computed.  The same order means that when
-//   S(b) is complete, PV(b - 3) is too, which bounds how far any barrier below
-//   can lag behind its waiter to one phase.  The first PV of a unit waits for
-//   the epilogue to have read the previous unit's O.
+//   QK(b) into S(b mod NS), then PV(b - NS + 1) from P(b - NS + 1).  QK(b)
+//   therefore waits for no softmax: the buffer it overwrites was last read by
+//   PV(b - NS), issued before it, and tcgen05 operations issued by one thread
+//   execute in order.  At NS = 3, while the softmax warps turn S(b) into P(b),
+//   S(b + 1) is already computed and S(b + 2) is being computed.  The same
+//   order means that when S(b) is complete, PV(b - NS) is too, which bounds
+//   how far any barrier below can lag behind its waiter to one phase.  The
+//   first PV of a unit waits for the epilogue to have read the previous
+//   unit's O.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <math.h>
