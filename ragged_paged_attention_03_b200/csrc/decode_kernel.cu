@@ -278,6 +278,9 @@ __device__ __forceinline__ void decode_body(const CUtensorMap &tm_k, const CUten
       m_run[nt][1] = mn1;
       const float p0 = ptx::ex2(x0 - mn0), p1 = ptx::ex2(x1 - mn1);
       const float p2 = ptx::ex2(x2 - mn0), p3 = ptx::ex2(x3 - mn1);
+      // l sums the fp32 weights: the max is updated every block, so the
+      // largest weight is exactly 1 and the bf16 rounding of the others
+      // moves O by far less than a bf16 step
       l_run[nt][0] = l_run[nt][0] * al0 + p0 + p2;
       l_run[nt][1] = l_run[nt][1] * al1 + p1 + p3;
 #pragma unroll

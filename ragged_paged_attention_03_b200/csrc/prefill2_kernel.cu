@@ -705,7 +705,7 @@ __global__ void __launch_bounds__(384, 1)
       const int n = t ? w.n_t[1] : w.n_t[0];
       const int rows_mine = t ? w.rows_t[1] : w.rows_t[0];
       const int rn = w.r0 + t * BM + row;        // new-token index of this row
-      float m = -INFINITY, l = 0.f;
+      float m = -INFINITY, l = 0.f, lr = 0.f;   // lr: the normaliser of O (below)
       for (int j = 0; j < n; ++j) {
         if (!__all_sync(0xffffffffu,
                         wait_bar2(&bars->s_full[t], (uint32_t)((gt + j) & 1), abort_flag, pb.err))) {
@@ -742,7 +742,8 @@ __global__ void __launch_bounds__(384, 1)
             mq[3] = ptx::fmax3(mq[3], x[i + 6], x[i + 7]);
           }
         }
-        const float mx = ptx::fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * scale_log2;
+        const float mraw = ptx::fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
+        const float mx = mraw * scale_log2;
         const float m_new = fmaxf(m, mx);
         const bool need = m != -INFINITY && m_new > m + kRescaleThreshold;
         float alpha = 1.f;
@@ -794,7 +795,16 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int k = 0; k < 4; ++k) ptx::f2_unpack(sp2[k], sp[2 * k], sp[2 * k + 1]);
         const float sum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+        // The PV MMA takes P rounded to bf16.  Under the lazy rescale the
+        // block's largest weight can be up to 2^8 (not exactly 1), and its
+        // rounding (relative 2^-9) moves O by up to 2^-9 |V| when one key
+        // dominates the row.  lr, the normaliser of O, therefore counts that
+        // weight as rounded, so that its rounding cancels in O / lr; the
+        // other weights keep the error of a kernel whose max weight is 1.
+        // l keeps the exact fp32 sum, for lse.
+        const float pmax = ptx::ex2(fmaf(mraw, scale_log2, neg_m));   // as the loop computed it
         l = l * alpha + sum;
+        lr = lr * alpha + (sum - (pmax - ptx::round_bf16(pmax)));
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
         ptx::mbar_arrive(&bars->p_full[t]);
@@ -807,7 +817,7 @@ __global__ void __launch_bounds__(384, 1)
         break;
       }
       ptx::tc_fence_after();
-      const float inv = 1.f / l;
+      const float inv = 1.f / lr;
       const bool store = row < rows_mine;
       __nv_bfloat16 *out =
           reinterpret_cast<__nv_bfloat16 *>(pb.out) + ((size_t)(w.tile.q_start + rn) * pb.hq + w.h) * D;

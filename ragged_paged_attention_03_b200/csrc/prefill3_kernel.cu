@@ -90,7 +90,9 @@ struct P3 {
   static constexpr int NSV = D == 128 ? (PAIR ? 4 : 2) : 2;
   static constexpr int kData = NQ * kQBytes + NSK * kKBytes + NSV * kVBytes;
   static constexpr int HK = BN / 2;               // keys of a block per softmax warpgroup
-  static constexpr int kStatFloats = 2 * 3 * BM;   // [unit parity][l of keys 0-63, l of keys 64-127, m][row]
+  // [unit parity][l of keys 0-63, l of keys 64-127, m, lr of keys 0-63, lr of keys 64-127][row]
+  // (l: sums of the fp32 weights, for lse; lr: the normalisers of O)
+  static constexpr int kStatFloats = 2 * 5 * BM;
   static constexpr int kRedFloats = 2 * 2 * BM;    // [exchange parity][warpgroup][row]: partial row maxima
   static constexpr int kSmem = 1024 + kData + (kStatFloats + kRedFloats) * 4 + 512;
   static constexpr uint32_t kTmemCols = 512;
@@ -636,7 +638,7 @@ __device__ __forceinline__ void softmax_loop(const Sync &sy, const Problem &pb, 
     const int ob = gu & 1;
     const int rn = w.my_r0 + row;                    // new-token index of this row
     const bool live = row < w.my_rows;
-    float m = -INFINITY, l = 0.f;
+    float m = -INFINITY, l = 0.f, lr = 0.f;   // lr: this half's share of the normaliser of O (below)
     for (int j = 0; j < w.nb; ++j, ++gb) {
       const int sb = gb % S::NS;
       const uint32_t tS = lane_base + (uint32_t)(sb * 128);
@@ -742,7 +744,16 @@ __device__ __forceinline__ void softmax_loop(const Sync &sy, const Problem &pb, 
 #pragma unroll
         for (int q = 0; q < 4; ++q) ptx::f2_unpack(sp2[q], sp[2 * q], sp[2 * q + 1]);
         const float sum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+        // The PV MMA takes P rounded to bf16.  Under the lazy rescale the
+        // largest weight of this half-block can be up to 2^8 (not exactly
+        // 1), and its rounding (relative 2^-9) moves O by up to 2^-9 |V|
+        // when one key dominates the row.  lr, the normaliser of O,
+        // therefore counts that weight as rounded, so that its rounding
+        // cancels in O / lr; the other weights keep the error of a kernel
+        // whose max weight is 1.  l keeps the exact fp32 sum, for lse.
+        const float pmax = ptx::ex2(fmaf(mine, scale_log2, neg_m));   // as the loop computed it
         l = l * alpha + sum;
+        lr = lr * alpha + (sum - (pmax - ptx::round_bf16(pmax)));
       }
       ptx::tmem_st_wait();
       ptx::tc_fence_before();
@@ -754,8 +765,9 @@ __device__ __forceinline__ void softmax_loop(const Sync &sy, const Problem &pb, 
       ok = false;
       break;
     }
-    stats[(ob * 3 + half) * S::BM + row] = l;
-    if (half == 0) stats[(ob * 3 + 2) * S::BM + row] = m;
+    stats[(ob * 5 + half) * S::BM + row] = l;
+    stats[(ob * 5 + 3 + half) * S::BM + row] = lr;
+    if (half == 0) stats[(ob * 5 + 2) * S::BM + row] = m;
     ptx::mbar_arrive(&bars->st_full[ob]);
     ++gu;
   }
@@ -780,15 +792,16 @@ __device__ __forceinline__ void epilogue_loop(const Sync &sy, const Problem &pb,
     if (!__all_sync(0xffffffffu, wait3<PAIR>(sy, &bars->o_full, (uint32_t)(gu & 1)))) break;
     if (!__all_sync(0xffffffffu, wait3<PAIR>(sy, &bars->st_full[ob], ph))) break;
     ptx::tc_fence_after();
-    const float l = stats[(ob * 3 + 0) * S::BM + row] + stats[(ob * 3 + 1) * S::BM + row];
-    const float m = stats[(ob * 3 + 2) * S::BM + row];
+    const float l = stats[(ob * 5 + 0) * S::BM + row] + stats[(ob * 5 + 1) * S::BM + row];
+    const float lr = stats[(ob * 5 + 3) * S::BM + row] + stats[(ob * 5 + 4) * S::BM + row];
+    const float m = stats[(ob * 5 + 2) * S::BM + row];
     ptx::mbar_arrive(&bars->st_free[ob]);
     // O a 32-column chunk at a time into registers, scaled by 1 / l and
     // stored; released after the last chunk (its next writer, the next
     // unit's first PV, is queued two blocks behind that unit's QKs)
     const bool store = row < w.my_rows;
     const int rn = w.my_r0 + row;
-    const float inv = store ? 1.f / l : 0.f;
+    const float inv = store ? 1.f / lr : 0.f;
     const uint64_t once = ptx::l2_evict_first_policy();   // outputs are written once: first out of L2
     uint4 *out = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(pb.out) +
                                            ((size_t)(w.tile.q_start + (store ? rn : 0)) * pb.hq + w.h) * S::D);

@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
     }
-    float m = -INFINITY, l = 0.f;
+    float m = -INFINITY, l = 0.f, lr = 0.f;   // lr: the normaliser of O (below)
     bool ok = true;
     for (int j = 0; j < nb; ++j) {
       const int b = j & 1;
@@ -427,7 +427,8 @@ __global__ void __launch_bounds__(192, 1)
           mq[3] = ptx::fmax3(mq[3], x[i + 6], x[i + 7]);
         }
       }
-      const float mx = ptx::fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * scale_log2;
+      const float mraw = ptx::fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
+      const float mx = mraw * scale_log2;
       const float m_new = fmaxf(m, mx);
       const bool need = m == -INFINITY ? false : (m_new > m + kRescaleThreshold);
       float alpha = 1.f;
@@ -479,8 +480,17 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
       for (int k = 0; k < 4; ++k) ptx::f2_unpack(sp2[k], spf[2 * k], spf[2 * k + 1]);
       const float sum = ((spf[0] + spf[1]) + (spf[2] + spf[3])) + ((spf[4] + spf[5]) + (spf[6] + spf[7]));
+      // The PV MMA takes P rounded to bf16.  Under the lazy rescale the
+      // block's largest weight can be up to 2^8 (not exactly 1), and its
+      // rounding (relative 2^-9) moves O by up to 2^-9 |V| when one key
+      // dominates the row.  lr, the normaliser of O, therefore counts that
+      // weight as rounded, so that its rounding cancels in O / lr; the
+      // other weights keep the error of a kernel whose max weight is 1.
+      // l keeps the exact fp32 sum, for lse.
+      const float pmax = ptx::ex2(fmaf(mraw, scale_log2, neg_m));   // as the loop computed it
       ptx::tmem_st_wait();
       l = l * alpha + sum;
+      lr = lr * alpha + (sum - (pmax - ptx::round_bf16(pmax)));
       ptx::tc_fence_before();
       ptx::mbar_arrive(&bars->p_full[b]);
     }
@@ -488,7 +498,7 @@ __global__ void __launch_bounds__(192, 1)
     if (ok && __all_sync(0xffffffffu, wait_bar(&bars->pv_done[(nb - 1) & 1], (uint32_t)(((nb - 1) >> 1) & 1),
                                                 abort_flag, pb.err))) {
       ptx::tc_fence_after();
-      const float inv = 1.f / l;
+      const float inv = 1.f / lr;
       const bool store = row < tile.rows;
       const uint64_t once = ptx::l2_evict_first_policy();   // written once: first out of L2
       __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(pb.out) +

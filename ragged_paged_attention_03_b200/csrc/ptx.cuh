@@ -147,6 +147,9 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return r;
 }
 
+// x rounded to bf16 (nearest even, as pack_bf16 does), as an fp32 value.
+__device__ __forceinline__ float round_bf16(float x) { return __uint_as_float(pack_bf16(x, 0.f) << 16); }
+
 // 2^x on the multi-function unit (approximate, flushes denormals).
 __device__ __forceinline__ float ex2(float x) {
   float y;

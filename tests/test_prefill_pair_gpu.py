@@ -51,6 +51,17 @@ def test_forced_prefill_kernel(oracle_mod, kernel_option, table, case):
     full_check(oracle_mod, prob)
 
 
+@pytest.mark.parametrize("kernel_option", list(KERNELS), ids=list(KERNELS.values()), indirect=True)
+@pytest.mark.parametrize("seed", [710, 711, 712, 714])
+def test_forced_dominant_key_after_context_block(oracle_mod, kernel_option, seed):
+    """The rows of test_parity_gpu's test_dominant_key_after_context_block on
+    the forced kernels: their row sums also take the bf16-rounded weights."""
+    ql, kv, hq, hkv, d, p, causal = SMALL[10]
+    prob = I.make_problem(ql, kv, num_q_heads=hq, num_kv_heads=hkv, head_dim=d, page_size=p,
+                          dtype=I.BF16, causal=causal, seed=seed, pool=1.5)
+    full_check(oracle_mod, prob)
+
+
 @pytest.mark.parametrize("kernel_option", [2, 1], ids=["pair", "one-tile"], indirect=True)
 @pytest.mark.parametrize("table,case", CASES_256, ids=[f"{t}{c}" for t, c in CASES_256])
 def test_forced_head_dim_256(oracle_mod, kernel_option, table, case):
