@@ -28,7 +28,8 @@
 //               through shared memory, each turns its half of S(b) into P(b)
 //               (bf16, back into S(b)'s columns: the A operand of the PV MMA)
 //               and keeps its share of the row sum
-//   warps 8-11  epilogue: O / l of a finished unit from TMEM to `out`, lse
+//   warps 8-11  epilogue: O / l of a finished unit from TMEM to `out`, lse;
+//               while a unit computes, four fifths of its cache update
 //   warp 12     TMA producer of Q tiles (two buffers) and K blocks of 128
 //               keys (context from cache pages, new tokens from k_new; rows
 //               without a valid key zeroed)
@@ -37,8 +38,8 @@
 //               that last read its stage (PV(b - 4) at head_dim 128), which
 //               is queued NS - 1 blocks behind its QK, so a producer shared
 //               with K would hold every K load back by as much
-//   warp 15     fused cache update: this CTA's share of the unit's new K/V
-//               rows copied into their page slots
+//   warp 15     fused cache update: a fifth of this CTA's share of each
+//               unit's new K/V rows copied into their page slots
 //
 // TMEM (512 columns, the same columns in both CTAs of a pair):
 //   head_dim 128: S(0) | S(1) | S(2) | O, 128 columns each (NS = 3);
@@ -540,15 +541,20 @@ __device__ __forceinline__ void produce(const Sync &sy, const Problem &pb, const
 }
 
 // --------------------------------------------------------- cache update
-// One warp copies this CTA's share of the new K/V rows of each unit into
-// their page slots: the G query heads of a KV head split the unit's rows,
-// and the two CTAs of a pair split each share.  Each lane keeps kBatch
-// 16-byte chunks (and their page-table entries) in flight before storing.
+// The new K/V rows of each unit are copied into their page slots by five
+// warps of the CTA: the cache-writer warp and the four epilogue warps (idle
+// while a unit computes).  The G query heads of a KV head split the unit's
+// rows, and the two CTAs of a pair split each share.  Warp wi of the five
+// takes every fifth group of 32 16-byte chunks; each lane keeps kBatch
+// chunks (and their page-table entries) in flight before storing.
+constexpr int kCacheWriters = 5;
+
 template <bool PAIR, int D>
-__device__ __forceinline__ void cache_update(const Problem &pb, const PrefillTile *tiles, int n_units, int rank) {
+__device__ __forceinline__ void cache_write_unit(const Problem &pb, const Unit3 &w, int rank, int wi) {
   using S = P3<PAIR, D>;
   if (!kCacheWrite) return;
-  constexpr int kBatch = 8;
+  constexpr int kBatch = 4;
+  constexpr int kStride = 32 * kCacheWriters;
   const int lane = threadIdx.x & 31;
   const int G = pb.hq / pb.hkv;
   constexpr int chunks = S::D / 8;
@@ -556,53 +562,59 @@ __device__ __forceinline__ void cache_update(const Problem &pb, const PrefillTil
   const __nv_bfloat16 *vn = reinterpret_cast<const __nv_bfloat16 *>(pb.v_new);
   __nv_bfloat16 *kc = reinterpret_cast<__nv_bfloat16 *>(pb.k_cache);
   __nv_bfloat16 *vc = reinterpret_cast<__nv_bfloat16 *>(pb.v_cache);
+  const int32_t *pt_row = pb.page_table + (size_t)w.tile.seq * pb.max_pages;
+  // rows of the unit: the item (pair) or this CTA's tile
+  const int u0 = PAIR ? w.tile.tile_row : w.my_r0;
+  const int un = PAIR ? w.tile.rows : w.my_rows;
+  const int gidx = w.h % G;
+  int ra = (gidx * un) / G, rb = ((gidx + 1) * un) / G;
+  if constexpr (PAIR) {
+    const int len = rb - ra;
+    const int a = ra + (rank * len) / 2, b = ra + ((rank + 1) * len) / 2;
+    ra = a;
+    rb = b;
+  }
+  const int total = (rb - ra) * chunks;
+  for (int base = wi * 32 + lane; base < total; base += kStride * kBatch) {
+    uint4 kq[kBatch], vq[kBatch];
+    int pgq[kBatch];
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+      const int idx = base + q * kStride;
+      if (idx < total) {
+        const int i = u0 + ra + idx / chunks;   // new-token index
+        const size_t src = ((size_t)(w.tile.q_start + i) * pb.hkv + w.hk) * S::D + (idx % chunks) * 8;
+        kq[q] = *reinterpret_cast<const uint4 *>(kn + src);
+        vq[q] = *reinterpret_cast<const uint4 *>(vn + src);
+        pgq[q] = pt_row[(w.c + i) / pb.p];
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+      const int idx = base + q * kStride;
+      if (idx >= total) continue;
+      const int i = u0 + ra + idx / chunks, ch = idx % chunks;
+      const int pos = w.c + i;
+      const int pg = pgq[q];
+      if (pg < 0 || pg >= pb.num_pages) {
+        if (ch == 0) atomicOr(pb.err, RPA_DEV_BAD_PAGE);
+        continue;
+      }
+      const size_t dst = (((size_t)pg * pb.p + pos % pb.p) * pb.hkv + w.hk) * S::D + ch * 8;
+      *reinterpret_cast<uint4 *>(kc + dst) = kq[q];
+      *reinterpret_cast<uint4 *>(vc + dst) = vq[q];
+    }
+  }
+}
+
+// The cache-writer warp's loop: its share (wi = 0) of every unit of the CTA.
+template <bool PAIR, int D>
+__device__ __forceinline__ void cache_update(const Problem &pb, const PrefillTile *tiles, int n_units, int rank) {
   for (int k = 0;; ++k) {
     const Unit3 w = make_unit3<PAIR>(tiles, unit_of<PAIR>(k), n_units, pb, rank);
     if (w.end) break;
     if (w.skip) continue;
-    const int32_t *pt_row = pb.page_table + (size_t)w.tile.seq * pb.max_pages;
-    // rows of the unit: the item (pair) or this CTA's tile
-    const int u0 = PAIR ? w.tile.tile_row : w.my_r0;
-    const int un = PAIR ? w.tile.rows : w.my_rows;
-    const int gidx = w.h % G;
-    int ra = (gidx * un) / G, rb = ((gidx + 1) * un) / G;
-    if constexpr (PAIR) {
-      const int len = rb - ra;
-      const int a = ra + (rank * len) / 2, b = ra + ((rank + 1) * len) / 2;
-      ra = a;
-      rb = b;
-    }
-    const int total = (rb - ra) * chunks;
-    for (int base = lane; base < total; base += 32 * kBatch) {
-      uint4 kq[kBatch], vq[kBatch];
-      int pgq[kBatch];
-#pragma unroll
-      for (int q = 0; q < kBatch; ++q) {
-        const int idx = base + q * 32;
-        if (idx < total) {
-          const int i = u0 + ra + idx / chunks;   // new-token index
-          const size_t src = ((size_t)(w.tile.q_start + i) * pb.hkv + w.hk) * S::D + (idx % chunks) * 8;
-          kq[q] = *reinterpret_cast<const uint4 *>(kn + src);
-          vq[q] = *reinterpret_cast<const uint4 *>(vn + src);
-          pgq[q] = pt_row[(w.c + i) / pb.p];
-        }
-      }
-#pragma unroll
-      for (int q = 0; q < kBatch; ++q) {
-        const int idx = base + q * 32;
-        if (idx >= total) continue;
-        const int i = u0 + ra + idx / chunks, ch = idx % chunks;
-        const int pos = w.c + i;
-        const int pg = pgq[q];
-        if (pg < 0 || pg >= pb.num_pages) {
-          if (ch == 0) atomicOr(pb.err, RPA_DEV_BAD_PAGE);
-          continue;
-        }
-        const size_t dst = (((size_t)pg * pb.p + pos % pb.p) * pb.hkv + w.hk) * S::D + ch * 8;
-        *reinterpret_cast<uint4 *>(kc + dst) = kq[q];
-        *reinterpret_cast<uint4 *>(vc + dst) = vq[q];
-      }
-    }
+    cache_write_unit<PAIR, D>(pb, w, rank, 0);
   }
 }
 
@@ -787,6 +799,8 @@ __device__ __forceinline__ void epilogue_loop(const Sync &sy, const Problem &pb,
     const Unit3 w = make_unit3<PAIR>(tiles, unit_of<PAIR>(k), n_units, pb, rank);
     if (w.end) break;
     if (w.skip) continue;
+    // this warp's share of the unit's cache update, while the unit computes
+    cache_write_unit<PAIR, D>(pb, w, rank, 1 + (warp & 3));
     const int ob = gu & 1;
     const uint32_t ph = (uint32_t)((gu >> 1) & 1);
     if (!__all_sync(0xffffffffu, wait3<PAIR>(sy, &bars->o_full, (uint32_t)(gu & 1)))) break;
