@@ -140,21 +140,6 @@ __device__ __forceinline__ Unit make_unit(const PrefillTile &tile, int u, const 
   return w;
 }
 
-// The next unit's Q tiles into L2 at the top of the current unit: their load
-// into shared memory waits for this unit's last QK, and would otherwise
-// start that late from DRAM.
-template <int D, int BM, int BN>
-__device__ __forceinline__ void prefetch_next_q(const PrefillTile &next, int u, int n_units, const Problem &pb,
-                                                const CUtensorMap &tm_q) {
-  if (u >= n_units || next.rows == 0) return;
-  const Unit n = make_unit<BM, BN>(next, u, pb);
-  for (int t = 0; t < 2; ++t) {
-    if (n.rows_t[t] == 0) continue;
-    for (int hh = 0; hh < D / 64; ++hh)
-      ptx::tma_prefetch_3d_elect(&tm_q, hh * 64, n.h, n.tile.q_start + n.r0 + t * BM);
-  }
-}
-
 // QK(t, gblk): S of tile t = Q_t K^T for K/V block gblk (K stage gblk % NSK).
 template <int D>
 __device__ __forceinline__ bool issue_qk(Bars2 *bars, volatile int *abort_flag, uint32_t *err, uint32_t tS,
@@ -316,7 +301,6 @@ __device__ __forceinline__ void produce_kv(Bars2 *bars, volatile int *abort_flag
     const Unit w = make_unit<BM, BN>(next, u, pb);
     next = load_tile(tiles, unit_of(r + 1), n_units, pb.hq);
     if (w.tile.rows == 0) break;   // end of a device-planned tile list
-    prefetch_next_q<D, BM, BN>(next, unit_of(r + 1), n_units, pb, tm_q);
     const int32_t *pt_row = pb.page_table + (size_t)w.tile.seq * pb.max_pages;
     // Q of both tiles, once the previous unit's QK MMAs are done with sQ
     if (uq > 0 && !wait_all(&bars->q_empty, (uint32_t)((uq - 1) & 1), abort_flag, pb.err)) break;
@@ -474,7 +458,6 @@ __device__ __forceinline__ void produce(Bars2 *bars, volatile int *abort_flag, c
     const Unit w = make_unit<BM, BN>(next, u, pb);
     next = load_tile(tiles, unit_of(r + 1), n_units, pb.hq);
     if (w.tile.rows == 0) break;   // end of a device-planned tile list
-    if (!IS_V) prefetch_next_q<D, BM, BN>(next, unit_of(r + 1), n_units, pb, *tm_q);
     const int32_t *pt_row = pb.page_table + (size_t)w.tile.seq * pb.max_pages;
     if (!IS_V) {
       // Q of both tiles, once the previous unit's QK MMAs are done with sQ

@@ -489,13 +489,6 @@ __device__ __forceinline__ void produce(const Sync &sy, const Problem &pb, const
     if (w.skip) continue;
     const int32_t *pt_row = pb.page_table + (size_t)w.tile.seq * pb.max_pages;
     if (!IS_V) {
-      // the next unit's Q rows into L2 now: their load into shared memory
-      // waits for a QK of this unit, and would otherwise start that late
-      // from DRAM
-      const Unit3 wn = make_unit3<PAIR>(tiles, unit_of<PAIR>(k + 1), n_units, pb, rank);
-      if (!wn.end && !wn.skip)
-        for (int hh = 0; hh < S::D / 64; ++hh)
-          ptx::tma_prefetch_3d_elect(tm_q, hh * 64, wn.h, wn.tile.q_start + wn.my_r0);
       // Q of this CTA's rows, once the unit that last used the buffer has
       // finished its QKs
       const int qb = gu % S::NQ;

@@ -76,16 +76,6 @@ __device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }
 
-// Prefetch of one 3-D box of a tensor into L2 (no shared memory, no
-// barrier), issued by one elected lane of the warp.
-__device__ __forceinline__ void tma_prefetch_3d_elect(const void *tmap, int32_t c0, int32_t c1, int32_t c2) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
-      "@e cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];\n\t}" ::"l"(tmap),
-      "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
-
 // 3-D tiled bulk-tensor load into shared memory, completion counted on `bar`.
 __device__ __forceinline__ void tma_load_3d(void *dst, const void *tmap, uint64_t *bar, int32_t c0,
                                             int32_t c1, int32_t c2) {
