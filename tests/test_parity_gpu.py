@@ -129,6 +129,29 @@ def test_decode_heavy_split_kv(oracle_mod, chunk):
         binding.rpa_set_option(binding.RPA_OPT_DECODE_CHUNK_BLOCKS, old)
 
 
+@pytest.mark.parametrize("chunk,inline", [(1, False), (16, True)])
+def test_decode_only_plan_in_or_beyond_launch_parameters(oracle_mod, chunk, inline):
+    """A decode-only batch whose work items fit in the launch parameters
+    (the inline plan, no upload) and the same batch cut into more items than
+    those hold (the plan uploaded to device memory): both paths against the
+    oracle."""
+    from ragged_paged_attention_03_b200 import binding
+    old = binding.rpa_set_option(binding.RPA_OPT_DECODE_CHUNK_BLOCKS, chunk)
+    try:
+        prob = I.make_problem([1] * 4, [4000, 5000, 3000, 3500], num_q_heads=16, num_kv_heads=2,
+                              head_dim=128, page_size=16, dtype=I.BF16, seed=23, pool=1.3)
+        d = binding.rpa_dims(num_q_heads=16, num_kv_heads=2, head_dim=128, page_size=16,
+                             num_pages=prob.k_cache.shape[0], max_pages_per_seq=prob.page_table.shape[1],
+                             total_q_tokens=prob.q.shape[0], dtype=binding.RPA_BF16)
+        info = binding.rpa_plan(np.asarray(prob.cu_q_lens, dtype=np.int32),
+                                np.asarray(prob.kv_lens, dtype=np.int32), prob.distribution, d)
+        assert (info.decode_items <= 900 and info.combine_rows <= 1800) == inline, \
+            (info.decode_items, info.combine_rows)
+        full_check(oracle_mod, prob)
+    finally:
+        binding.rpa_set_option(binding.RPA_OPT_DECODE_CHUNK_BLOCKS, old)
+
+
 @pytest.mark.parametrize("loaders", [1, 2])
 @pytest.mark.parametrize("case", [4, 5, 6, 7, 8])
 def test_prefill_loader_builds(oracle_mod, loaders, case):
