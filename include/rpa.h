@@ -192,9 +192,13 @@ enum {
                                       kernel (default 0) */
   RPA_OPT_DISABLE_PREFILL_TC = 2,  /* 1: prefill sequences use the generic
                                       kernel instead of tensor cores */
-  RPA_OPT_PREFILL_SMS = 3,         /* most CTAs (SMs) of the head_dim <= 128
-                                      prefill kernel in a concurrent mixed
-                                      batch (default 0: one per SM) */
+  RPA_OPT_PREFILL_SMS = 3,         /* SMs of the prefill kernel in a
+                                      concurrent mixed batch: k > 0 at most
+                                      k; 0 (default) sized from the plan, the
+                                      prefill's estimated share of the two
+                                      kernels' SM-time (x1.2, even, at least
+                                      16; rpa_forward_device: every SM);
+                                      < 0 every SM */
   RPA_OPT_CONCURRENT_MIXED = 4,    /* >= 0 (default 0): the prefill and the
                                       decode work of a mixed batch run
                                       concurrently, prefill on a

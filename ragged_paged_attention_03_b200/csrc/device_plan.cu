@@ -428,7 +428,7 @@ extern "C" RPA_API int rpa_forward_device(const void *q, const void *k_new, cons
       pstream = ss->side;
     }
     if (e == cudaSuccess && L.cap_tiles > 0)
-      e = launch_prefill_any(pb, a.tiles, (int)L.cap_tiles, (int)prefill_sms(), false, pstream);
+      e = launch_prefill_any(pb, a.tiles, (int)L.cap_tiles, (int)std::max<int64_t>(0, prefill_sms()), false, pstream);
     const cudaError_t ej = ss ? cudaEventRecord(ss->join, pstream) : cudaSuccess;
     if (e == cudaSuccess) e = ej;
     if (e == cudaSuccess && L.cap_items > 0)

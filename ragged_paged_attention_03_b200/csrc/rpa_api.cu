@@ -441,6 +441,41 @@ cudaError_t traced(int kind, cudaStream_t stream, F &&launch) {
 }
 
 
+// SMs for the prefill kernel of a batch with both kinds of rows when
+// RPA_OPT_PREFILL_SMS is 0.  A decode SM moves a fixed share of HBM
+// bandwidth and a prefill SM does a fixed share of the MMAs, so the step
+// lasts about as long as the two kernels' summed SM-time over the GPU, and
+// the schedule matters at the end: an SM that takes prefill units first and
+// finishes them late, when the decode work is done, idles the rest.  So the
+// prefill gets its estimated share of the SM-time (1.2 times it, even, at
+// least 16 SMs) and the decode CTAs take the other SMs from the start.  The
+// per-SM rates are this kernel set's measured ones on B200; only their ratio
+// matters.
+int auto_prefill_ctas(const HostPlan &hp, const Problem &pb, int sms) {
+  constexpr double kPrefillFlopsPerSm128 = 6.0e12, kPrefillFlopsPerSm256 = 8.6e12;
+  constexpr double kDecodeBytesPerSm = 41.0e9;
+  double blocks = 0;   // 128-row x 128-key score blocks of every tile half (one query head)
+  for (const PrefillTile &t : hp.prefill) {
+    const int n_ctx = (t.kv_len - t.q_len + 127) / 128;
+    for (int h = 0; h * 128 < t.rows; ++h) {
+      const int rows = std::min(128, t.rows - h * 128);
+      const int new_end = pb.causal ? t.tile_row + h * 128 + rows : t.q_len;
+      blocks += n_ctx + (new_end + 127) / 128;
+    }
+  }
+  const double flops = blocks * 128.0 * 128.0 * 4.0 * pb.d * pb.hq;
+  double kv_blocks = 0;   // 16-token blocks of K/V read by the decode items
+  for (const DecodeItem &it : hp.decode) kv_blocks += it.blk_end - it.blk_begin;
+  for (const DecodeItem &it : hp.decode_packed) kv_blocks += it.blk_end - it.blk_begin;
+  const double bytes = kv_blocks * 16.0 * pb.hkv * pb.d * 2.0 * 2.0;
+  const double tp = flops / (pb.d > 128 ? kPrefillFlopsPerSm256 : kPrefillFlopsPerSm128);
+  const double td = bytes / kDecodeBytesPerSm;
+  if (tp <= 0 || td <= 0) return 0;
+  int n = (int)std::ceil(1.2 * sms * tp / (tp + td));
+  n = std::max(16, n + (n & 1));
+  return n >= sms ? 0 : n;   // 0: one per SM
+}
+
 // The kernels of one planned call, queued on `stream` (the caller holds
 // ws.mu).  A batch with both prefill and decode work runs them
 // concurrently: the compute-bound prefill kernel on the high-priority side
@@ -463,7 +498,7 @@ cudaError_t launch_kernels(DeviceWs &ws, const HostPlan &hp, const int32_t *dev_
   int prefill_ctas = 0;
   if (mixed) {
     const int64_t k = g_opt_prefill_sms.load();
-    prefill_ctas = k > 0 ? (int)std::min<int64_t>(k, ws.sms) : 0;   // 0: one per SM
+    prefill_ctas = k > 0 ? (int)std::min<int64_t>(k, ws.sms) : k == 0 ? auto_prefill_ctas(hp, pb, ws.sms) : 0;
     pstream = ws.side;
     if (cudaEventRecord(fork, stream) != cudaSuccess || cudaStreamWaitEvent(pstream, fork, 0) != cudaSuccess)
       return cudaErrorUnknown;
