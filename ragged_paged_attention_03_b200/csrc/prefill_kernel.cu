@@ -28,6 +28,10 @@
 // Keys are ordered as context blocks [0, c) followed by new-token blocks
 // starting at c, so with BN = 128 the causal diagonal of a 128-row tile is
 // exactly one block.
+//
+// At head_dim 256 this kernel is selectable (RPA_OPT_PREFILL_KERNEL = 1); the
+// default there is the CTA-pair kernel of prefill3_kernel.cu, whose MMAs
+// outpace this one-tile-per-CTA design.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <math.h>
