@@ -566,6 +566,7 @@ __device__ __forceinline__ void cache_update(const Problem pb, const PrefillTile
   const __nv_bfloat16 *vn = reinterpret_cast<const __nv_bfloat16 *>(pb.v_new);
   __nv_bfloat16 *kc = reinterpret_cast<__nv_bfloat16 *>(pb.k_cache);
   __nv_bfloat16 *vc = reinterpret_cast<__nv_bfloat16 *>(pb.v_cache);
+  const uint64_t once = ptx::l2_evict_first_policy();
   PrefillTile next = load_tile(tiles, unit_of(0), n_units, pb.hq);
   for (int r = 0, u = unit_of(0); u < n_units; u = unit_of(++r)) {
     const Unit w = make_unit<BM, BN>(next, u, pb);
@@ -585,8 +586,10 @@ __device__ __forceinline__ void cache_update(const Problem pb, const PrefillTile
       }
       const size_t src = ((size_t)(w.tile.q_start + i) * pb.hkv + w.hk) * D + ch * 8;
       const size_t dst = (((size_t)pg * pb.p + pos % pb.p) * pb.hkv + w.hk) * D + ch * 8;
-      *reinterpret_cast<uint4 *>(kc + dst) = *reinterpret_cast<const uint4 *>(kn + src);
-      *reinterpret_cast<uint4 *>(vc + dst) = *reinterpret_cast<const uint4 *>(vn + src);
+      // written once and not read again by this launch: first out of L2,
+      // ahead of the K/V blocks that other query heads still read
+      ptx::st_global_hint(kc + dst, *reinterpret_cast<const uint4 *>(kn + src), once);
+      ptx::st_global_hint(vc + dst, *reinterpret_cast<const uint4 *>(vn + src), once);
     }
   }
 }

@@ -563,6 +563,7 @@ __device__ __forceinline__ void cache_write_unit(const Problem &pb, const Unit3 
   __nv_bfloat16 *kc = reinterpret_cast<__nv_bfloat16 *>(pb.k_cache);
   __nv_bfloat16 *vc = reinterpret_cast<__nv_bfloat16 *>(pb.v_cache);
   const int32_t *pt_row = pb.page_table + (size_t)w.tile.seq * pb.max_pages;
+  const uint64_t once = ptx::l2_evict_first_policy();
   // rows of the unit: the item (pair) or this CTA's tile
   const int u0 = PAIR ? w.tile.tile_row : w.my_r0;
   const int un = PAIR ? w.tile.rows : w.my_rows;
@@ -601,8 +602,10 @@ __device__ __forceinline__ void cache_write_unit(const Problem &pb, const Unit3 
         continue;
       }
       const size_t dst = (((size_t)pg * pb.p + pos % pb.p) * pb.hkv + w.hk) * S::D + ch * 8;
-      *reinterpret_cast<uint4 *>(kc + dst) = kq[q];
-      *reinterpret_cast<uint4 *>(vc + dst) = vq[q];
+      // written once and not read again by this launch: first out of L2,
+      // ahead of the K/V blocks that other query heads still read
+      ptx::st_global_hint(kc + dst, kq[q], once);
+      ptx::st_global_hint(vc + dst, vq[q], once);
     }
   }
 }
