@@ -124,6 +124,9 @@ __device__ __forceinline__ void decode_body(const CUtensorMap &tm_k, const CUten
   // Queues the TMA copies of this warp's it-th block into its stage
   // (lane 0 only).  Boxes holding no cached position are skipped; their rows
   // are filled when the block is consumed.
+  // every K/V byte is read by this CTA alone, once: first out of L2, so that
+  // a prefill kernel running beside it keeps its reused K/V blocks there
+  const uint64_t once = ptx::l2_evict_first_policy();
   auto issue = [&](int k) {
     const int b = it.blk_begin + (PACK ? k : warp + kWarps * k);
     if (b >= it.blk_end) return;
@@ -148,8 +151,8 @@ __device__ __forceinline__ void decode_body(const CUtensorMap &tm_k, const CUten
       const int row = pg * P + (pos % P);
 #pragma unroll
       for (int h = 0; h < S::kHalves; ++h) {
-        ptx::tma_load_3d(sk + h * S::kTile + r0 * 128, &tm_k, &my_bars[st], h * 64, hk, row);
-        ptx::tma_load_3d(sv + h * S::kTile + r0 * 128, &tm_v, &my_bars[st], h * 64, hk, row);
+        ptx::tma_load_3d_hint(sk + h * S::kTile + r0 * 128, &tm_k, &my_bars[st], h * 64, hk, row, once);
+        ptx::tma_load_3d_hint(sv + h * S::kTile + r0 * 128, &tm_v, &my_bars[st], h * 64, hk, row, once);
       }
     }
   };
