@@ -141,3 +141,42 @@ def test_head_shard_job_value():
     assert bench.value_of("decode_128", w, 1.0, 4) == pytest.approx(4 * 1e9 / 1e-3 / 1e9)
     assert bench.rank_work(work, 4, "replicas") is work
     assert bench.value_of("mixed_96d_4c", work, 1.0, 4) == pytest.approx(4 * 1000 / 1e-3)
+
+
+def test_traffic_records_only_for_the_captured_source_and_kernel(tmp_path, monkeypatch):
+    """A DRAM-traffic record is reported only while its kernel source is the
+    one that was captured and the run uses the captured kernel option."""
+    import hashlib
+    import json
+    src = tmp_path / "k.cu"
+    src.write_text("kernel v1\n")
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    rec = {"prefill/w": {"dram_bytes_per_launch": 123, "source": "k.cu",
+                         "source_sha256": hashlib.sha256(b"kernel v1\n").hexdigest(),
+                         "prefill_kernel_option": 0}}
+    (prof / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "PREFILL_KERNEL_OPTION", 0)
+    assert bench.traffic_for("prefill", "w") == 123
+    assert bench.traffic_for("decode", "w") is None
+    monkeypatch.setattr(bench, "PREFILL_KERNEL_OPTION", 2)
+    assert bench.traffic_for("prefill", "w") is None
+    monkeypatch.setattr(bench, "PREFILL_KERNEL_OPTION", 0)
+    src.write_text("kernel v2\n")
+    assert bench.traffic_for("prefill", "w") is None
+
+
+def test_committed_traffic_records_match_their_sources():
+    """Every committed record names an existing kernel source; a record whose
+    source has changed since the capture is reported as null by the bench
+    (this only lists them, it does not fail: recapturing needs a GPU)."""
+    import hashlib
+    import json
+    recs = json.load(open(os.path.join(bench.ROOT, "profiles", "traffic.json")))
+    for key, rec in recs.items():
+        path = os.path.join(bench.ROOT, rec["source"])
+        assert os.path.exists(path), key
+        assert rec["dram_bytes_per_launch"] > 0, key
+        fresh = hashlib.sha256(open(path, "rb").read()).hexdigest() == rec["source_sha256"]
+        print(key, "current" if fresh else "stale (reported as null)")
