@@ -501,6 +501,10 @@ def dist_setup(args, backend="nccl"):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1 and args.impl == "ours":
         import datetime
+        if backend == "nccl":
+            # each rank's GPU before the group forms, so that NCCL (and the
+            # first barrier) binds this rank to its own device
+            torch.cuda.set_device(local)
         torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return world, rank, local
 
