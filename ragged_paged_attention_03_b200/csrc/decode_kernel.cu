@@ -48,7 +48,7 @@ struct DecodeShape {
   static constexpr int kHalves = D / 64;                  // 128-byte column tiles
   static constexpr int kTile = 16 * 128;                  // 16 rows x 64 bf16, swizzled
   static constexpr int kStage = 2 * kHalves * kTile;      // K tiles then V tiles
-  static constexpr int kStages = D == 64 ? 6 : 3;
+  static constexpr int kStages = D == 64 ? 6 : (D == 128 ? 2 : 3);
   static constexpr int kRing = kWarps * kStages * kStage;
   static constexpr int kSmem = 1024 + kRing + kMaxItemPages * 4 + kWarps * kStages * 8;
 };
